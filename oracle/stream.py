@@ -70,10 +70,12 @@ class _Frame:
     __slots__ = ("k_special", "v_special", "k_patch", "v_patch")
 
     def __init__(self, k, v, ns):
-        self.k_special = k[:ns].copy()
-        self.v_special = v[:ns].copy()
-        self.k_patch = k[ns:].copy()
-        self.v_patch = v[ns:].copy()
+        # Views, not copies: a stream that cycles through a few distinct data
+        # frames shares their memory.  Callers must not modify the arrays.
+        self.k_special = k[:ns]
+        self.v_special = v[:ns]
+        self.k_patch = k[ns:]
+        self.v_patch = v[ns:]
 
 
 class FrameStream:

@@ -1,0 +1,435 @@
+// Paged attention on the sm_100a tensor cores (tcgen05 MMA, TMEM accumulators,
+// TMA page gathers).
+//
+// What it computes ("How Paged KV Cache Attention Enables ~20 FPS Streaming
+// Inference in LingBot-Map", Sec. FlashInfer Paged-Kernel Integration and
+// Sec. Step-by-Step Streaming Inference, step 4; "How the Paged KV Cache
+// Attention Mechanism Enables Long Sequence Inference in LingBot-Map",
+// Sec. FlashInfer Kernel Execution): for one frame's queries, softmax over
+// every visible token of the stream -- the pages listed by the visible page
+// table, each full except the last (last_page_len valid tokens) -- with no
+// causal mask, read straight from the page pool.
+//
+// Work item = (stream, head, 128-row query tile, KV chunk).  One CTA per item:
+//   warp 4      TMA producer: Q tile once, then K and V tiles of 128 tokens,
+//               gathered page by page through the visible table (a page of
+//               page_size tokens is ceil(page_size/128) tiles; rows past the
+//               page end are zero-filled by TMA and masked).
+//   warp 5      MMA issuer (one thread) and TMEM owner:
+//                 S_j = Q K_j^T      (SS MMA, fp32 into TMEM, double buffered)
+//                 O  += P_j V_j      (TS MMA: P_j read from TMEM, V_j from smem)
+//   warps 0-3   softmax: thread r owns query row r = TMEM lane r; reads S_j,
+//               online softmax in the log2 domain with a lazy rescale of O
+//               (only when the running max grows by more than 2^8), writes
+//               P_j as 16-bit pairs over the first half of S_j's columns,
+//               then the epilogue (O / l, LSE).
+// S_{j+1} is computed while the softmax works on S_j.  Split-KV chunks write
+// fp32 partials and LSE; a merge kernel combines them.
+
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+
+#include "sm100_primitives.cuh"
+#include "svt_internal.h"
+
+namespace svt {
+namespace {
+
+using namespace sm100;
+
+constexpr int kThreads = 192;
+constexpr int kTmemCols = 512;
+constexpr uint64_t kWaitLimitNs = 2000000000ull;   // 2 s
+constexpr float kRescaleThreshold = 8.0f;          // log2 units
+
+template <int D>
+struct Cfg {
+  static constexpr int kRegions = D / 64;                      // 64-feature swizzle columns
+  static constexpr uint32_t kTileBytes = kTileN * D * 2;       // one K or V (or Q) tile
+  static constexpr uint32_t kRegionBytes = kTileN * 128;       // 128 rows x 128 bytes
+  static constexpr int kStages = D == 64 ? 4 : 2;
+  static constexpr uint32_t kQOff = 0;
+  static constexpr uint32_t kKOff = kTileM * D * 2;
+  static constexpr uint32_t kVOff = kKOff + kStages * kTileBytes;
+  static constexpr uint32_t kBarOff = kVOff + kStages * kTileBytes;
+  // barriers: q_full, k_full[S], k_empty[S], v_full[S], v_empty[S], s_full[2], p_full[2],
+  // o_done[2] (PV_j commits to o_done[j&1]), drain ; then tmem base word and abort flag
+  static constexpr int kNumBars = 1 + 4 * kStages + 2 + 2 + 2 + 1;
+  static constexpr uint32_t kMiscOff = kBarOff + kNumBars * 8;
+  static constexpr uint32_t kSmemBytes = kMiscOff + 16 + 1024;   // + alignment slack
+  static constexpr uint32_t kTmemS0 = 0, kTmemS1 = 128, kTmemO = 256;
+};
+
+struct Item {
+  int st, head, qtile, chunk, t_begin, n_tiles;
+};
+
+__device__ __forceinline__ Item decode_item(const AttnParams& p) {
+  Item it;
+  int st = 0;
+  while (st + 1 < p.n_streams && (int)blockIdx.x >= p.s[st + 1].item_off) ++st;
+  const StreamPlan& sp = p.s[st];
+  const int local = blockIdx.x - sp.item_off;
+  it.st = st;
+  it.qtile = local % sp.qtiles;
+  const int rest = local / sp.qtiles;
+  it.chunk = rest % sp.chunks;
+  it.head = rest / sp.chunks;
+  const int t0 = (int)((int64_t)it.chunk * sp.tiles / sp.chunks);
+  const int t1 = (int)((int64_t)(it.chunk + 1) * sp.tiles / sp.chunks);
+  it.t_begin = t0;
+  it.n_tiles = t1 - t0;
+  return it;
+}
+
+// Tile g of a stream's KV sequence -> (position in the visible table, tile in page, valid rows).
+__device__ __forceinline__ void tile_coords(const StreamPlan& sp, int P, int g, int& page_pos,
+                                            int& t, int& valid) {
+  const int tpp = (P + kTileN - 1) / kTileN;
+  const int full = (sp.n_pages - 1) * tpp;
+  int page_tokens;
+  if (g < full) {
+    page_pos = g / tpp;
+    t = g % tpp;
+    page_tokens = P;
+  } else {
+    page_pos = sp.n_pages - 1;
+    t = g - full;
+    page_tokens = sp.lpl;
+  }
+  valid = min(kTileN, page_tokens - t * kTileN);
+}
+
+template <int D, bool BF16>
+__global__ void __launch_bounds__(kThreads, 1)
+    attn_sm100_kernel(const __grid_constant__ CUtensorMap tmap_q,
+                      const __grid_constant__ CUtensorMap tmap_kv,
+                      const __grid_constant__ AttnParams p) {
+  using C = Cfg<D>;
+  using T = typename std::conditional<BF16, __nv_bfloat16, __half>::type;
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw = smem_addr(smem_raw);
+  const uint32_t base = (raw + 1023u) & ~1023u;
+  uint8_t* gbase = smem_raw + (base - raw);
+  const uint32_t sQ = base + C::kQOff;
+  const uint32_t sK = base + C::kKOff;
+  const uint32_t sV = base + C::kVOff;
+  const uint32_t bars = base + C::kBarOff;
+  auto q_full = [&]() { return bars; };
+  auto k_full = [&](int s) { return bars + 8u * (1 + s); };
+  auto k_empty = [&](int s) { return bars + 8u * (1 + C::kStages + s); };
+  auto v_full = [&](int s) { return bars + 8u * (1 + 2 * C::kStages + s); };
+  auto v_empty = [&](int s) { return bars + 8u * (1 + 3 * C::kStages + s); };
+  auto s_full = [&](int b) { return bars + 8u * (1 + 4 * C::kStages + b); };
+  auto p_full = [&](int b) { return bars + 8u * (3 + 4 * C::kStages + b); };
+  auto o_done = [&](int b) { return bars + 8u * (5 + 4 * C::kStages + b); };
+  const uint32_t drain = bars + 8u * (7 + 4 * C::kStages);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(gbase + C::kMiscOff);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(gbase + C::kMiscOff + 4);
+
+  const int warp = threadIdx.x / 32;
+  const int lane = threadIdx.x % 32;
+  const Item it = decode_item(p);
+  const StreamPlan& sp = p.s[it.st];
+  const int n = it.n_tiles;
+
+  if (threadIdx.x == 0) {
+    *abort_flag = 0;
+    mbar_init(q_full(), 1);
+    for (int s = 0; s < C::kStages; ++s) {
+      mbar_init(k_full(s), 1);
+      mbar_init(k_empty(s), 1);
+      mbar_init(v_full(s), 1);
+      mbar_init(v_empty(s), 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(s_full(b), 1);
+      mbar_init(p_full(b), 128);
+    }
+    mbar_init(o_done(0), 1);
+    mbar_init(o_done(1), 1);
+    mbar_init(drain, 1);
+    fence_barrier_init();
+    fence_proxy_async_shared();
+  }
+  if (warp == 5) {
+    tmem_alloc(smem_addr(tmem_slot), kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  auto fail = [&]() {
+    *abort_flag = 1;
+    atomicOr(p.err, kErrWaitLimit);
+  };
+
+  if (warp == 4) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      tma_prefetch_desc(&tmap_q);
+      tma_prefetch_desc(&tmap_kv);
+      mbar_arrive_expect_tx(q_full(), kTileM * D * 2);
+      for (int r = 0; r < C::kRegions; ++r)
+        tma_load_3d(sQ + r * C::kRegionBytes, &tmap_q, q_full(), r * 64, it.head,
+                    sp.q_off + it.qtile * kTileM);
+      int issued = 0;
+      for (int j = 0; j < n; ++j) {
+        int page_pos, t, valid;
+        tile_coords(sp, p.P, it.t_begin + j, page_pos, t, valid);
+        int page = p.indices[sp.page_off + page_pos];
+        if (page < 0 || page >= p.max_pages) {
+          atomicOr(p.err, kErrPageId);
+          page = 0;
+        }
+        const int c4 = (int)(p.block_page_base + page);
+        const int s = j % C::kStages;
+        const uint32_t ph = (j / C::kStages) & 1;
+        if (!mbar_wait(k_empty(s), ph ^ 1, abort_flag, kWaitLimitNs)) { fail(); break; }
+        mbar_arrive_expect_tx(k_full(s), C::kTileBytes);
+        for (int r = 0; r < C::kRegions; ++r)
+          tma_load_5d(sK + s * C::kTileBytes + r * C::kRegionBytes, &tmap_kv, k_full(s), r * 64,
+                      it.head, t * kTileN, 0, c4);
+        if (!mbar_wait(v_empty(s), ph ^ 1, abort_flag, kWaitLimitNs)) { fail(); issued = j + 1; break; }
+        mbar_arrive_expect_tx(v_full(s), C::kTileBytes);
+        for (int r = 0; r < C::kRegions; ++r)
+          tma_load_5d(sV + s * C::kTileBytes + r * C::kRegionBytes, &tmap_kv, v_full(s), r * 64,
+                      it.head, t * kTileN, 1, c4);
+        issued = j + 1;
+      }
+      if (*abort_flag) {
+        // Let the copies already in flight land before the CTA exits.
+        mbar_wait(q_full(), 0, nullptr, kWaitLimitNs);
+        for (int j = max(0, issued - C::kStages); j < issued; ++j) {
+          const int s = j % C::kStages;
+          const uint32_t ph = (j / C::kStages) & 1;
+          mbar_wait(k_full(s), ph, nullptr, kWaitLimitNs);
+          mbar_wait(v_full(s), ph, nullptr, kWaitLimitNs);
+        }
+      }
+    }
+  } else if (warp == 5) {
+    // ---------------------------------------------------------- MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t idS = idesc_f16(kTileM, kTileN, BF16, false);
+      constexpr uint32_t idO = idesc_f16(kTileM, D, BF16, true);
+      bool ok = mbar_wait(q_full(), 0, abort_flag, kWaitLimitNs);
+      if (!ok) fail();
+      tc_fence_after();
+      auto issue_s = [&](int j) -> bool {
+        const int s = j % C::kStages;
+        if (!mbar_wait(k_full(s), (j / C::kStages) & 1, abort_flag, kWaitLimitNs)) return false;
+        tc_fence_after();
+        const uint32_t d = tmem + ((j & 1) ? C::kTmemS1 : C::kTmemS0);
+        const uint32_t kb = sK + s * C::kTileBytes;
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t off = (kk / 4) * C::kRegionBytes + (kk % 4) * 32;
+          mma_ss(d, desc_sw128(sQ + off, 16, 1024), desc_sw128(kb + off, 16, 1024), idS,
+                 kk > 0 ? 1u : 0u);
+        }
+        mma_commit(k_empty(s));
+        mma_commit(s_full(j & 1));
+        return true;
+      };
+      if (ok && n > 0) ok = issue_s(0);
+      for (int j = 0; ok && j < n; ++j) {
+        if (j + 1 < n && !(ok = issue_s(j + 1))) break;
+        if (!(ok = mbar_wait(p_full(j & 1), (j >> 1) & 1, abort_flag, kWaitLimitNs))) break;
+        tc_fence_after();
+        const int s = j % C::kStages;
+        const uint32_t vb = sV + s * C::kTileBytes;
+        const uint32_t a = tmem + ((j & 1) ? C::kTmemS1 : C::kTmemS0);
+#pragma unroll
+        for (int kk = 0; kk < kTileN / 16; ++kk)
+          mma_ts(tmem + C::kTmemO, a + kk * 8, desc_sw128(vb + kk * 2048, C::kRegionBytes, 1024),
+                 idO, (j > 0 || kk > 0) ? 1u : 0u);
+        mma_commit(v_empty(s));
+        mma_commit(o_done(j & 1));
+      }
+      if (!ok) fail();
+      // Drain: every MMA issued above has completed once `drain` flips.
+      mma_commit(drain);
+      mbar_wait(drain, 0, nullptr, kWaitLimitNs);
+    }
+  } else {
+    // ------------------------------------------------------ softmax warps
+    // Every tcgen05.ld/st below is executed by all 32 lanes of the warp: the
+    // branches around them are warp-uniform.  Barrier phases: S_j completes
+    // only after PV_{j-2} (in-order MMA pipe), so when PV_{j-1} is awaited on
+    // o_done[(j-1)&1] that barrier is at most one phase behind.
+    const int row = threadIdx.x;                          // 0..127 == TMEM lane
+    const uint32_t lane_addr = tmem + ((uint32_t)(warp * 32) << 16);
+    const float sl2 = p.scale_log2;
+    constexpr unsigned kAll = 0xffffffffu;
+    float m = -INFINITY, l = 0.f;
+    bool ok = true;
+    for (int j = 0; j < n; ++j) {
+      const int b = j & 1;
+      ok = __all_sync(kAll, mbar_wait(s_full(b), (j >> 1) & 1, abort_flag, kWaitLimitNs));
+      if (!ok) break;
+      tc_fence_after();
+      int page_pos, t, valid;
+      tile_coords(sp, p.P, it.t_begin + j, page_pos, t, valid);
+      const uint32_t sb = lane_addr + (b ? C::kTmemS1 : C::kTmemS0);
+      uint32_t sr[4][32];
+#pragma unroll
+      for (int c = 0; c < 4; ++c) tmem_ld32(sb + c * 32, sr[c]);
+      tmem_wait_ld();
+      float mx = -INFINITY;
+#pragma unroll
+      for (int c = 0; c < 4; ++c)
+#pragma unroll
+        for (int i = 0; i < 32; ++i)
+          if (c * 32 + i < valid) mx = fmaxf(mx, __uint_as_float(sr[c][i]));
+      mx *= sl2;
+      if (j == 0) {
+        m = mx;
+      } else if (__any_sync(kAll, mx > m + kRescaleThreshold)) {
+        // O holds the sum over earlier tiles scaled by 2^-m: move it to the new max.
+        ok = __all_sync(kAll, mbar_wait(o_done((j - 1) & 1), ((j - 1) >> 1) & 1, abort_flag,
+                                        kWaitLimitNs));
+        if (!ok) break;
+        tc_fence_after();
+        const float mnew = fmaxf(m, mx);
+        const float alpha = ex2(m - mnew);
+        l *= alpha;
+#pragma unroll
+        for (int c = 0; c < D / 32; ++c) {
+          uint32_t o[32];
+          tmem_ld32(lane_addr + C::kTmemO + c * 32, o);
+          tmem_wait_ld();
+#pragma unroll
+          for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
+          tmem_st32(lane_addr + C::kTmemO + c * 32, o);
+        }
+        m = mnew;
+      }
+      const float neg_m = -m;
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        uint32_t pk[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          const int col = c * 32 + 2 * i;
+          const float p0 = col < valid ? ex2(fmaf(__uint_as_float(sr[c][2 * i]), sl2, neg_m)) : 0.f;
+          const float p1 =
+              col + 1 < valid ? ex2(fmaf(__uint_as_float(sr[c][2 * i + 1]), sl2, neg_m)) : 0.f;
+          l += p0 + p1;
+          if constexpr (BF16) {
+            __nv_bfloat162 h2 = __floats2bfloat162_rn(p0, p1);
+            pk[i] = *reinterpret_cast<uint32_t*>(&h2);
+          } else {
+            __half2 h2 = __floats2half2_rn(p0, p1);
+            pk[i] = *reinterpret_cast<uint32_t*>(&h2);
+          }
+        }
+        tmem_st16(sb + c * 16, pk);
+      }
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive(p_full(b));
+    }
+    if (ok && n > 0)
+      ok = __all_sync(kAll, mbar_wait(o_done((n - 1) & 1), ((n - 1) >> 1) & 1, abort_flag,
+                                      kWaitLimitNs));
+    if (!ok) fail();
+    tc_fence_after();
+    if (ok && n > 0) {
+      const int r = it.qtile * kTileM + row;
+      const bool store = r < sp.nq;
+      const float inv = 1.f / l;
+      const int grow = sp.q_off + (store ? r : 0);
+      const float lse = (m + __log2f(l)) * 0.69314718055994531f;
+      if (sp.chunks == 1) {
+        T* orow = static_cast<T*>(p.out) + ((size_t)grow * p.H + it.head) * D;
+#pragma unroll
+        for (int c = 0; c < D / 32; ++c) {
+          uint32_t o[32];
+          tmem_ld32(lane_addr + C::kTmemO + c * 32, o);
+          tmem_wait_ld();
+          uint32_t pk[16];
+#pragma unroll
+          for (int i = 0; i < 16; ++i) {
+            const float a0 = __uint_as_float(o[2 * i]) * inv;
+            const float a1 = __uint_as_float(o[2 * i + 1]) * inv;
+            if constexpr (BF16) {
+              __nv_bfloat162 h2 = __floats2bfloat162_rn(a0, a1);
+              pk[i] = *reinterpret_cast<uint32_t*>(&h2);
+            } else {
+              __half2 h2 = __floats2half2_rn(a0, a1);
+              pk[i] = *reinterpret_cast<uint32_t*>(&h2);
+            }
+          }
+          if (store) {
+            uint4* dst = reinterpret_cast<uint4*>(orow + c * 32);
+#pragma unroll
+            for (int v = 0; v < 4; ++v)
+              dst[v] = make_uint4(pk[4 * v], pk[4 * v + 1], pk[4 * v + 2], pk[4 * v + 3]);
+          }
+        }
+        if (store && p.lse) p.lse[(size_t)grow * p.H + it.head] = lse;
+      } else {
+        const size_t wrow = ((size_t)it.chunk * p.ws_rows + grow) * p.H + it.head;
+        float4* dst = reinterpret_cast<float4*>(p.ws_o + wrow * D);
+#pragma unroll
+        for (int c = 0; c < D / 32; ++c) {
+          uint32_t o[32];
+          tmem_ld32(lane_addr + C::kTmemO + c * 32, o);
+          tmem_wait_ld();
+          if (store) {
+#pragma unroll
+            for (int v = 0; v < 8; ++v)
+              dst[c * 8 + v] = make_float4(__uint_as_float(o[4 * v]) * inv,
+                                           __uint_as_float(o[4 * v + 1]) * inv,
+                                           __uint_as_float(o[4 * v + 2]) * inv,
+                                           __uint_as_float(o[4 * v + 3]) * inv);
+          }
+        }
+        if (store) p.ws_lse[wrow] = lse;
+      }
+    }
+    tc_fence_before();
+  }
+  __syncthreads();
+  if (warp == 5) {
+    tc_fence_after();
+    tmem_dealloc(tmem, kTmemCols);
+  }
+}
+
+template <int D, bool BF16>
+cudaError_t launch_t(const AttnParams& p, const void* tq, const void* tkv, cudaStream_t s) {
+  using C = Cfg<D>;
+  auto kern = attn_sm100_kernel<D, BF16>;
+  static bool configured = false;
+  if (!configured) {
+    cudaError_t e =
+        cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
+    if (e != cudaSuccess) return e;
+    configured = true;
+  }
+  CUtensorMap mq, mkv;
+  memcpy(&mq, tq, sizeof(mq));
+  memcpy(&mkv, tkv, sizeof(mkv));
+  kern<<<p.total_items, kThreads, C::kSmemBytes, s>>>(mq, mkv, p);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_attn_sm100(const AttnParams& p, const void* tmap_q, const void* tmap_kv,
+                              int dtype, cudaStream_t s) {
+  if (p.total_items == 0) return cudaSuccess;
+  const bool bf16 = dtype == SVT_BF16;
+  if (p.D == 64) return bf16 ? launch_t<64, true>(p, tmap_q, tmap_kv, s)
+                             : launch_t<64, false>(p, tmap_q, tmap_kv, s);
+  if (p.D == 128) return bf16 ? launch_t<128, true>(p, tmap_q, tmap_kv, s)
+                              : launch_t<128, false>(p, tmap_q, tmap_kv, s);
+  return cudaErrorInvalidValue;
+}
+
+}  // namespace svt

@@ -1,0 +1,911 @@
+// Host side of the streaming paged KV-cache library: the C ABI, the page
+// allocator with its free lists, the device page-table mirror, the planner
+// and the launches.
+//
+// The allocator follows the two-stream design of the pages:
+//  * patch stream: one page per frame, handed out from the front of a FIFO
+//    free list; the first scale_frames pages of a stream are permanent scale
+//    pages, later ones enter a sliding window of sliding_window frames and
+//    are returned to the back of the free list when they leave it.
+//    ("How LingBot-Map Uses KV Caching for Efficient Streaming Inference",
+//    Sec. Sliding-Window Eviction Strategy; "How FlashInfer's Paged KV Cache
+//    Attention Outperforms SDPA Fallback in Streaming Inference", Sec.
+//    Two-Stream Design.)
+//  * special stream: num_special tokens per frame packed continuously over
+//    pages of the same size, never evicted (same sections).
+//  * deferred eviction and rollback of the provisional frame ("How LingBot-Map
+//    Uses KV Caching ...", Sec. Flow-Based Keyframe Selection): rollback puts
+//    the pages back at the FRONT of their free lists so that the allocator
+//    state is exactly the state before the append.
+//
+// Device state kept by the library: a mirror of each stream's scale list,
+// window ring and special-page list, written by the block-0 append kernel
+// (page ids travel as kernel arguments, no host->device copies), from which
+// the builder kernel assembles the visible page table.
+
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
+#include <algorithm>
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+#include <cstdlib>
+#include <cstring>
+#include <deque>
+#include <mutex>
+#include <queue>
+#include <string>
+#include <vector>
+
+#include "svt_internal.h"
+
+using namespace svt;
+
+namespace {
+
+thread_local std::string g_err;
+
+int fail(int code, const char* fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof(buf), fmt, ap);
+  va_end(ap);
+  g_err = buf;
+  return code;
+}
+
+int cuda_fail(cudaError_t e, const char* what) {
+  return fail(SVT_ECUDA, "%s: %s", what, cudaGetErrorString(e));
+}
+
+int elem_size(int dtype) { return dtype == SVT_FP32 ? 4 : 2; }
+
+struct StreamState {
+  std::vector<int> scale;          // scale pages, frame order
+  std::deque<int> window;          // window pages, oldest -> newest
+  int ring_head = 0;               // device ring slot of window.front()
+  std::vector<int> special_pages;  // fill order
+  int64_t special_tokens = 0;
+  int64_t frame_count = 0;
+  bool defer = false;
+  bool has_prov = false;           // last frame is provisional
+  bool prov_scale = false;
+  int prov_new_sp = 0;             // special pages opened by the provisional frame
+  int blocks_done = 0;             // blocks that appended the current frame
+  int cur_patch = -1;              // pages of the current frame (for blocks > 0)
+  int cur_sp_off0 = 0;
+  int cur_n_sp = 0;
+  int cur_sp[kMaxSpecialSpan] = {0};
+};
+
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  });
+  return fn;
+}
+
+}  // namespace
+
+struct svt_cache {
+  // shape and options
+  int max_pages = 0, P = 0, H = 0, D = 0, W = 0, S = 0;
+  int L = 1, ns = 6, n_streams = 1, dtype = SVT_BF16, elem = 2;
+  int patch_pages = 0, max_qo = 0, max_splits = 16, rope_grid = 0;
+  float rope_theta = 100.f;
+  bool host_only = false;
+  bool debug_kv = false;
+  int num_sms = 148;
+  char* pool = nullptr;
+
+  // allocator
+  std::deque<int> patch_free, special_free;
+  std::vector<int> init_patch, init_special;
+  std::vector<StreamState> st;
+  bool dirty = true;       // state changed since the last table build
+  uint64_t version = 0;    // bumps on every build
+
+  // plan
+  bool plan_valid = false;
+  uint64_t plan_version = 0;
+  int total_rows = 0;
+  bool any_split = false;
+  AttnParams attn{};
+  SimtParams simt{};
+  svt_plan_info info{};
+
+  // device memory (one allocation)
+  void* dmem = nullptr;
+  int* d_scale = nullptr;
+  int* d_ring = nullptr;
+  int* d_special = nullptr;
+  int* d_indptr = nullptr;
+  int* d_indices = nullptr;
+  int* d_lpl = nullptr;
+  unsigned* d_err = nullptr;
+  float* d_ws_o = nullptr;
+  float* d_ws_lse = nullptr;
+  char* d_qrope = nullptr;
+  float2* d_rope_tab = nullptr;
+  int ring_cap = 1, sp_cap = 0, indices_cap = 0;
+
+  alignas(64) CUtensorMap tmap_kv;
+  bool has_tmap = false;
+  alignas(64) CUtensorMap tmap_q;
+  const void* tmap_q_ptr = nullptr;
+  int tmap_q_rows = -1;
+};
+
+namespace {
+
+size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+int page_valid_tokens_last(const svt_cache* c, const StreamState& s) {
+  if (!s.special_pages.empty()) return int((s.special_tokens - 1) % c->P) + 1;
+  if (!s.scale.empty() || !s.window.empty()) return c->P;
+  return 0;
+}
+
+int n_visible_pages(const StreamState& s) {
+  return int(s.scale.size() + s.window.size() + s.special_pages.size());
+}
+
+void mark_dirty(svt_cache* c) {
+  c->dirty = true;
+  c->plan_valid = false;
+}
+
+int check_stream(const svt_cache* c, int stream) {
+  if (!c) return fail(SVT_EINVAL, "null cache");
+  if (stream < 0 || stream >= c->n_streams)
+    return fail(SVT_EINVAL, "stream %d out of range [0,%d)", stream, c->n_streams);
+  return SVT_OK;
+}
+
+void debug_stats(const svt_cache* c, int stream, const char* when) {
+  if (!c->debug_kv) return;
+  const StreamState& s = c->st[stream];
+  fprintf(stderr,
+          "[svt] %s stream=%d frame_count=%lld scale_pages=%zu live_pages=%zu free_pages=%zu "
+          "special_tokens=%lld\n",
+          when, stream, (long long)s.frame_count, s.scale.size(), s.window.size(),
+          c->patch_free.size(), (long long)s.special_tokens);
+}
+
+int encode_kv_map(svt_cache* c) {
+  auto enc = tensor_map_encoder();
+  if (!enc) return fail(SVT_ECUDA, "cuTensorMapEncodeTiled entry point unavailable");
+  const cuuint64_t e = c->elem;
+  cuuint64_t dims[5] = {(cuuint64_t)c->D, (cuuint64_t)c->H, (cuuint64_t)c->P, 2,
+                        (cuuint64_t)c->L * (cuuint64_t)c->max_pages};
+  cuuint64_t strides[4] = {c->D * e, (cuuint64_t)c->H * c->D * e,
+                           (cuuint64_t)c->P * c->H * c->D * e,
+                           2ull * c->P * c->H * c->D * e};
+  cuuint32_t box[5] = {64, 1, (cuuint32_t)kTileN, 1, 1};
+  cuuint32_t estr[5] = {1, 1, 1, 1, 1};
+  CUresult r = enc(&c->tmap_kv,
+                   c->dtype == SVT_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16
+                                        : CU_TENSOR_MAP_DATA_TYPE_FLOAT16,
+                   5, c->pool, dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                   CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(SVT_ECUDA, "cuTensorMapEncodeTiled(pool) failed: %d", (int)r);
+  c->has_tmap = true;
+  return SVT_OK;
+}
+
+int encode_q_map(svt_cache* c, const void* q, int rows) {
+  if (c->tmap_q_ptr == q && c->tmap_q_rows == rows) return SVT_OK;
+  auto enc = tensor_map_encoder();
+  if (!enc) return fail(SVT_ECUDA, "cuTensorMapEncodeTiled entry point unavailable");
+  const cuuint64_t e = c->elem;
+  cuuint64_t dims[3] = {(cuuint64_t)c->D, (cuuint64_t)c->H, (cuuint64_t)rows};
+  cuuint64_t strides[2] = {c->D * e, (cuuint64_t)c->H * c->D * e};
+  cuuint32_t box[3] = {64, 1, (cuuint32_t)kTileM};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = enc(&c->tmap_q,
+                   c->dtype == SVT_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16
+                                        : CU_TENSOR_MAP_DATA_TYPE_FLOAT16,
+                   3, const_cast<void*>(q), dims, strides, box, estr,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(SVT_ECUDA, "cuTensorMapEncodeTiled(q) failed: %d", (int)r);
+  c->tmap_q_ptr = q;
+  c->tmap_q_rows = rows;
+  return SVT_OK;
+}
+
+void fill_rope_table(const svt_cache* c, std::vector<float2>& tab) {
+  // (cos, sin) of pos * theta^(-2i/m), m = D/2, i < m/2, pos < grid; double precision.
+  const int m = c->D / 2, half = m / 2;
+  tab.resize((size_t)c->rope_grid * half);
+  for (int pos = 0; pos < c->rope_grid; ++pos)
+    for (int i = 0; i < half; ++i) {
+      double ang = pos * std::pow((double)c->rope_theta, -2.0 * i / m);
+      tab[(size_t)pos * half + i] = make_float2((float)std::cos(ang), (float)std::sin(ang));
+    }
+}
+
+// ------------------------------------------------------------------ planner
+// Estimated makespan (us) of a list-scheduled launch: items are handed to the
+// SMs in blockIdx order as SMs become free.
+double simulate(const std::vector<double>& item_cost, int num_sms) {
+  std::priority_queue<double, std::vector<double>, std::greater<double>> sm;
+  for (int i = 0; i < num_sms; ++i) sm.push(0.0);
+  double end = 0;
+  for (double cst : item_cost) {
+    double t = sm.top();
+    sm.pop();
+    t += cst;
+    end = std::max(end, t);
+    sm.push(t);
+  }
+  return end;
+}
+
+}  // namespace
+
+// =================================================================== C ABI
+extern "C" {
+
+const char* svt_last_error(void) { return g_err.c_str(); }
+
+void svt_default_opts(svt_cache_opts* o) {
+  if (!o) return;
+  std::memset(o, 0, sizeof(*o));
+  o->num_blocks = 1;
+  o->num_special = 6;
+  o->num_streams = 1;
+  o->dtype = SVT_BF16;
+  o->max_splits = 16;
+  o->rope_theta = 100.f;
+}
+
+size_t svt_pool_bytes(int max_pages, int page_size, int H, int D, const svt_cache_opts* opts) {
+  svt_cache_opts o;
+  if (opts) o = *opts; else svt_default_opts(&o);
+  if (max_pages <= 0 || page_size <= 0 || H <= 0 || D <= 0 || o.num_blocks <= 0) return 0;
+  if (o.dtype < SVT_BF16 || o.dtype > SVT_FP32) return 0;
+  return (size_t)o.num_blocks * max_pages * 2 * page_size * H * D * elem_size(o.dtype);
+}
+
+int svt_create_cache(int max_pages, int page_size, int H, int D, int sliding_window,
+                     int scale_frames, const svt_cache_opts* opts, svt_cache** out) {
+  if (!out) return fail(SVT_EINVAL, "out is NULL");
+  *out = nullptr;
+  svt_cache_opts o;
+  if (opts) o = *opts; else svt_default_opts(&o);
+  if (o.num_blocks <= 0) o.num_blocks = 1;
+  if (o.num_streams <= 0) o.num_streams = 1;
+  if (o.max_splits <= 0) o.max_splits = 16;
+  if (o.rope_theta <= 0.f) o.rope_theta = 100.f;
+  if (max_pages <= 0 || page_size <= 0 || H <= 0 || D <= 0)
+    return fail(SVT_EINVAL, "max_pages, page_size, H, D must be positive");
+  if (sliding_window < 0 || scale_frames < 0)
+    return fail(SVT_EINVAL, "sliding_window and scale_frames must be >= 0");
+  if (o.num_special < 0 || o.num_special > page_size)
+    return fail(SVT_EINVAL, "num_special must be in [0, page_size]");
+  if (o.num_streams > SVT_MAX_STREAMS)
+    return fail(SVT_EINVAL, "num_streams > %d", SVT_MAX_STREAMS);
+  if (o.dtype < SVT_BF16 || o.dtype > SVT_FP32) return fail(SVT_EINVAL, "bad dtype");
+  if (o.max_splits > 64) return fail(SVT_EINVAL, "max_splits > 64");
+  if (D % 32 != 0 || D > 256) return fail(SVT_EINVAL, "D must be a multiple of 32, <= 256");
+  const int need_patch = o.num_streams * (scale_frames + sliding_window + 1);
+  const int patch_pages = o.patch_pages > 0 ? o.patch_pages : need_patch;
+  if (patch_pages < need_patch)
+    return fail(SVT_EINVAL, "patch_pages %d < num_streams*(scale_frames+sliding_window+1) = %d",
+                patch_pages, need_patch);
+  if (patch_pages >= max_pages)
+    return fail(SVT_EINVAL, "max_pages %d leaves no special pages after %d patch pages",
+                max_pages, patch_pages);
+  if (o.rope_grid < 0 || (o.rope_grid > 0 && o.rope_grid * o.rope_grid != page_size))
+    return fail(SVT_EINVAL, "rope_grid^2 must equal page_size");
+  if ((int64_t)o.num_blocks * max_pages >= (1ll << 31))
+    return fail(SVT_EINVAL, "num_blocks*max_pages too large");
+  if (!o.host_only) {
+    if (!o.pool) return fail(SVT_EINVAL, "opts->pool is NULL (allocate svt_pool_bytes)");
+    if (reinterpret_cast<uintptr_t>(o.pool) % 256)
+      return fail(SVT_EINVAL, "pool must be 256-byte aligned");
+    if (o.dtype != SVT_FP32 && !(D == 64 || D == 128))
+      return fail(SVT_EINVAL, "tensor-core path supports D in {64, 128}");
+    if ((size_t)H * D * elem_size(o.dtype) % 16)
+      return fail(SVT_EINVAL, "H*D*elem must be a multiple of 16 bytes");
+  }
+
+  svt_cache* c = new (std::nothrow) svt_cache();
+  if (!c) return fail(SVT_EINVAL, "out of host memory");
+  c->max_pages = max_pages;
+  c->P = page_size;
+  c->H = H;
+  c->D = D;
+  c->W = sliding_window;
+  c->S = scale_frames;
+  c->L = o.num_blocks;
+  c->ns = o.num_special;
+  c->n_streams = o.num_streams;
+  c->dtype = o.dtype;
+  c->elem = elem_size(o.dtype);
+  c->patch_pages = patch_pages;
+  c->max_qo = o.max_qo_len > 0 ? o.max_qo_len : o.num_streams * (o.num_special + page_size);
+  c->max_splits = o.max_splits;
+  c->rope_grid = o.rope_grid;
+  c->rope_theta = o.rope_theta;
+  c->host_only = o.host_only != 0;
+  c->pool = static_cast<char*>(o.pool);
+  const char* dbg = std::getenv("SVT_DEBUG_KV");
+  c->debug_kv = dbg && dbg[0] == '1';
+  c->ring_cap = sliding_window + 1;
+  c->sp_cap = max_pages - patch_pages;
+  c->indices_cap = o.num_streams * (scale_frames + sliding_window + 1) + c->sp_cap;
+  for (int i = 0; i < patch_pages; ++i) c->init_patch.push_back(i);
+  for (int i = patch_pages; i < max_pages; ++i) c->init_special.push_back(i);
+  c->st.resize(o.num_streams);
+  for (auto& s : c->st) s.blocks_done = c->L;
+  c->patch_free.assign(c->init_patch.begin(), c->init_patch.end());
+  c->special_free.assign(c->init_special.begin(), c->init_special.end());
+
+  if (!c->host_only) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e == cudaSuccess) e = cudaDeviceGetAttribute(&c->num_sms, cudaDevAttrMultiProcessorCount, dev);
+    if (e != cudaSuccess) { delete c; return cuda_fail(e, "cudaDeviceGetAttribute"); }
+    const int ns_ = c->n_streams;
+    size_t off = 0;
+    auto carve = [&](size_t bytes) { size_t at = off; off = align_up(off + bytes, 256); return at; };
+    size_t o_scale = carve(sizeof(int) * ns_ * std::max(1, c->S));
+    size_t o_ring = carve(sizeof(int) * ns_ * c->ring_cap);
+    size_t o_special = carve(sizeof(int) * ns_ * std::max(1, c->sp_cap));
+    size_t o_indptr = carve(sizeof(int) * (ns_ + 1));
+    size_t o_indices = carve(sizeof(int) * c->indices_cap);
+    size_t o_lpl = carve(sizeof(int) * ns_);
+    size_t o_err = carve(sizeof(unsigned));
+    size_t o_ws_o = carve(sizeof(float) * (size_t)c->max_splits * c->max_qo * H * D);
+    size_t o_ws_lse = carve(sizeof(float) * (size_t)c->max_splits * c->max_qo * H);
+    size_t o_qrope = c->rope_grid ? carve((size_t)c->max_qo * H * D * c->elem) : 0;
+    std::vector<float2> tab;
+    if (c->rope_grid) fill_rope_table(c, tab);
+    size_t o_tab = c->rope_grid ? carve(sizeof(float2) * tab.size()) : 0;
+    e = cudaMalloc(&c->dmem, off);
+    if (e != cudaSuccess) { delete c; return cuda_fail(e, "cudaMalloc(library state)"); }
+    char* b = static_cast<char*>(c->dmem);
+    c->d_scale = reinterpret_cast<int*>(b + o_scale);
+    c->d_ring = reinterpret_cast<int*>(b + o_ring);
+    c->d_special = reinterpret_cast<int*>(b + o_special);
+    c->d_indptr = reinterpret_cast<int*>(b + o_indptr);
+    c->d_indices = reinterpret_cast<int*>(b + o_indices);
+    c->d_lpl = reinterpret_cast<int*>(b + o_lpl);
+    c->d_err = reinterpret_cast<unsigned*>(b + o_err);
+    c->d_ws_o = reinterpret_cast<float*>(b + o_ws_o);
+    c->d_ws_lse = reinterpret_cast<float*>(b + o_ws_lse);
+    if (c->rope_grid) {
+      c->d_qrope = b + o_qrope;
+      c->d_rope_tab = reinterpret_cast<float2*>(b + o_tab);
+    }
+    e = cudaMemset(c->dmem, 0, off);
+    if (e == cudaSuccess && c->rope_grid)
+      e = cudaMemcpy(c->d_rope_tab, tab.data(), sizeof(float2) * tab.size(), cudaMemcpyHostToDevice);
+    if (e != cudaSuccess) { cudaFree(c->dmem); delete c; return cuda_fail(e, "cache init"); }
+    if (c->dtype != SVT_FP32) {
+      int r = encode_kv_map(c);
+      if (r) { cudaFree(c->dmem); delete c; return r; }
+    }
+  }
+  *out = c;
+  return SVT_OK;
+}
+
+int svt_destroy_cache(svt_cache* c) {
+  if (!c) return SVT_OK;
+  if (c->dmem) cudaFree(c->dmem);
+  delete c;
+  return SVT_OK;
+}
+
+int svt_reset(svt_cache* c) {
+  if (!c) return fail(SVT_EINVAL, "null cache");
+  for (auto& s : c->st) {
+    s = StreamState();
+    s.blocks_done = c->L;
+  }
+  c->patch_free.assign(c->init_patch.begin(), c->init_patch.end());
+  c->special_free.assign(c->init_special.begin(), c->init_special.end());
+  mark_dirty(c);
+  return SVT_OK;
+}
+
+int svt_set_free_lists(svt_cache* c, const int32_t* patch_ids, int n_patch,
+                       const int32_t* special_ids, int n_special) {
+  if (!c) return fail(SVT_EINVAL, "null cache");
+  for (const auto& s : c->st)
+    if (s.frame_count) return fail(SVT_ESTATE, "free lists can only be set on an empty cache");
+  if (n_patch != c->patch_pages || n_special != c->max_pages - c->patch_pages || !patch_ids ||
+      (n_special && !special_ids))
+    return fail(SVT_EINVAL, "free lists must list every page of their class");
+  std::vector<char> seen(c->max_pages, 0);
+  for (int i = 0; i < n_patch; ++i) {
+    int p = patch_ids[i];
+    if (p < 0 || p >= c->patch_pages || seen[p]) return fail(SVT_EINVAL, "bad patch page id %d", p);
+    seen[p] = 1;
+  }
+  for (int i = 0; i < n_special; ++i) {
+    int p = special_ids[i];
+    if (p < c->patch_pages || p >= c->max_pages || seen[p])
+      return fail(SVT_EINVAL, "bad special page id %d", p);
+    seen[p] = 1;
+  }
+  c->init_patch.assign(patch_ids, patch_ids + n_patch);
+  c->init_special.assign(special_ids, special_ids + n_special);
+  return svt_reset(c);
+}
+
+int svt_append_frame(svt_cache* c, int block, int stream, const void* k, const void* v,
+                     svt_stream_t cs) {
+  if (int r = check_stream(c, stream)) return r;
+  if (block < 0 || block >= c->L) return fail(SVT_EINVAL, "block %d out of range", block);
+  if (c->host_only) {
+    if (k || v) return fail(SVT_EINVAL, "host-only cache takes no k/v");
+  } else if (!k || !v) {
+    return fail(SVT_EINVAL, "k and v must be device pointers");
+  }
+  StreamState& s = c->st[stream];
+  const int P = c->P, ns = c->ns;
+  AppendParams ap{};
+  if (block == 0) {
+    if (s.blocks_done != c->L)
+      return fail(SVT_ESTATE, "block 0 of a new frame before blocks %d..%d of the previous one",
+                  s.blocks_done, c->L - 1);
+    if (s.has_prov)
+      return fail(SVT_ESTATE, "previous frame is provisional: execute_deferred_eviction or "
+                              "rollback_last_frame first");
+    if ((int)s.window.size() > c->W)
+      return fail(SVT_ESTATE, "window holds %zu > sliding_window frames: call evict_frames "
+                              "after each append", s.window.size());
+    // specials: tokens [n0, n0+ns) of the stream's special sequence
+    const int64_t n0 = s.special_tokens;
+    const int first_pg = int(n0 / P);
+    const int last_pg = ns ? int((n0 + ns - 1) / P) : first_pg - 1;
+    const int n_new = std::max(0, last_pg + 1 - (int)s.special_pages.size());
+    const int n_touch = ns ? last_pg - first_pg + 1 : 0;
+    if (n_touch > kMaxSpecialSpan) return fail(SVT_EINVAL, "special tokens span too many pages");
+    if (c->patch_free.empty()) return fail(SVT_ENOPAGES, "patch free list is empty");
+    if ((int)c->special_free.size() < n_new) return fail(SVT_ENOPAGES, "special free list is empty");
+    if ((int64_t)s.special_pages.size() + n_new > c->sp_cap)
+      return fail(SVT_ENOPAGES, "special page capacity exhausted");
+    // allocate (no failure after this point except a launch error, which is rolled back)
+    const int page = c->patch_free.front();
+    c->patch_free.pop_front();
+    int new_sp[kMaxSpecialSpan];
+    for (int i = 0; i < n_new; ++i) {
+      new_sp[i] = c->special_free.front();
+      c->special_free.pop_front();
+      s.special_pages.push_back(new_sp[i]);
+    }
+    const bool is_scale = (int)s.scale.size() < c->S;
+    int slot_index;
+    if (is_scale) {
+      slot_index = (int)s.scale.size();
+      s.scale.push_back(page);
+    } else {
+      slot_index = (s.ring_head + (int)s.window.size()) % c->ring_cap;
+      s.window.push_back(page);
+    }
+    s.special_tokens += ns;
+    s.frame_count += 1;
+    s.has_prov = s.defer;
+    s.prov_scale = is_scale;
+    s.prov_new_sp = n_new;
+    s.blocks_done = 0;
+    s.cur_patch = page;
+    s.cur_sp_off0 = ns ? int(n0 % P) : 0;
+    s.cur_n_sp = n_touch;
+    for (int i = 0; i < n_touch; ++i) s.cur_sp[i] = s.special_pages[first_pg + i];
+    mark_dirty(c);
+    if (!c->host_only) {
+      ap.mirror_patch = (is_scale ? c->d_scale + (size_t)stream * std::max(1, c->S)
+                                  : c->d_ring + (size_t)stream * c->ring_cap) + slot_index;
+      ap.mirror_special = c->d_special + (size_t)stream * std::max(1, c->sp_cap) +
+                          (s.special_pages.size() - n_new);
+      ap.n_new_sp = n_new;
+      for (int i = 0; i < n_new; ++i) ap.new_sp[i] = new_sp[i];
+    }
+  } else if (s.blocks_done != block) {
+    return fail(SVT_ESTATE, "block %d appended out of order (expected block %d)", block,
+                s.blocks_done == c->L ? 0 : s.blocks_done);
+  }
+  if (!c->host_only) {
+    ap.pool_block = c->pool + (size_t)block * c->max_pages * 2 * P * c->H * c->D * c->elem;
+    ap.k = static_cast<const char*>(k);
+    ap.v = static_cast<const char*>(v);
+    ap.ns = ns;
+    ap.P = P;
+    ap.H = c->H;
+    ap.D = c->D;
+    ap.elem = c->elem;
+    ap.patch_page = s.cur_patch;
+    ap.sp_off0 = s.cur_sp_off0;
+    ap.n_sp = s.cur_n_sp;
+    for (int i = 0; i < s.cur_n_sp; ++i) ap.sp_pages[i] = s.cur_sp[i];
+    ap.rope_tab = c->rope_grid ? c->d_rope_tab : nullptr;
+    ap.rope_grid = c->rope_grid;
+    cudaError_t e = launch_append(ap, c->dtype, reinterpret_cast<cudaStream_t>(cs));
+    if (e != cudaSuccess) {
+      if (block == 0) {  // undo the allocation so that a failed call changes nothing
+        s.has_prov = true;
+        svt_rollback_last_frame(c, stream);
+        s.has_prov = false;
+      }
+      return cuda_fail(e, "append kernel launch");
+    }
+  }
+  s.blocks_done = block + 1;
+  if (block == 0) debug_stats(c, stream, "append");
+  return SVT_OK;
+}
+
+int svt_evict_frames(svt_cache* c, int stream) {
+  if (int r = check_stream(c, stream)) return r;
+  StreamState& s = c->st[stream];
+  if (s.has_prov) return SVT_OK;  // eviction deferred
+  bool changed = false;
+  while ((int)s.window.size() > c->W) {
+    c->patch_free.push_back(s.window.front());
+    s.window.pop_front();
+    s.ring_head = (s.ring_head + 1) % c->ring_cap;
+    changed = true;
+  }
+  if (changed) {
+    mark_dirty(c);
+    debug_stats(c, stream, "evict");
+  }
+  return SVT_OK;
+}
+
+int svt_set_defer_eviction(svt_cache* c, int stream, int on) {
+  if (int r = check_stream(c, stream)) return r;
+  c->st[stream].defer = on != 0;
+  return SVT_OK;
+}
+
+int svt_execute_deferred_eviction(svt_cache* c, int stream) {
+  if (int r = check_stream(c, stream)) return r;
+  StreamState& s = c->st[stream];
+  if (!s.has_prov) return fail(SVT_ESTATE, "no provisional frame to accept");
+  s.has_prov = false;
+  return svt_evict_frames(c, stream);
+}
+
+int svt_rollback_last_frame(svt_cache* c, int stream) {
+  if (int r = check_stream(c, stream)) return r;
+  StreamState& s = c->st[stream];
+  if (!s.has_prov) return fail(SVT_ESTATE, "no provisional frame to roll back");
+  for (int i = 0; i < s.prov_new_sp; ++i) {
+    c->special_free.push_front(s.special_pages.back());
+    s.special_pages.pop_back();
+  }
+  int page;
+  if (s.prov_scale) {
+    page = s.scale.back();
+    s.scale.pop_back();
+  } else {
+    page = s.window.back();
+    s.window.pop_back();
+  }
+  c->patch_free.push_front(page);
+  s.special_tokens -= c->ns;
+  s.frame_count -= 1;
+  s.has_prov = false;
+  s.prov_new_sp = 0;
+  s.blocks_done = c->L;
+  mark_dirty(c);
+  debug_stats(c, stream, "rollback");
+  return SVT_OK;
+}
+
+int svt_get_cache_stats(const svt_cache* c, int stream, svt_stats* out) {
+  if (int r = check_stream(c, stream)) return r;
+  if (!out) return fail(SVT_EINVAL, "out is NULL");
+  const StreamState& s = c->st[stream];
+  out->frame_count = s.frame_count;
+  out->scale_pages = (int64_t)s.scale.size();
+  out->live_pages = (int64_t)s.window.size();
+  out->free_pages = (int64_t)c->patch_free.size();
+  out->special_tokens = s.special_tokens;
+  return SVT_OK;
+}
+
+int svt_get_page_table(const svt_cache* c, int32_t* indptr, int32_t* indices,
+                       int32_t* last_page_len, int capacity, int* n_pages) {
+  if (!c) return fail(SVT_EINVAL, "null cache");
+  int total = 0;
+  for (const auto& s : c->st) total += n_visible_pages(s);
+  if (n_pages) *n_pages = total;
+  if (!indptr || !last_page_len || (total && !indices)) return fail(SVT_EINVAL, "null output");
+  if (capacity < total) return fail(SVT_EINVAL, "capacity %d < %d entries", capacity, total);
+  int at = 0;
+  for (int i = 0; i < c->n_streams; ++i) {
+    const StreamState& s = c->st[i];
+    indptr[i] = at;
+    for (int p : s.scale) indices[at++] = p;
+    for (int p : s.window) indices[at++] = p;
+    for (int p : s.special_pages) indices[at++] = p;
+    last_page_len[i] = page_valid_tokens_last(c, s);
+  }
+  indptr[c->n_streams] = at;
+  return SVT_OK;
+}
+
+int svt_build_visible_page_table(svt_cache* c, svt_stream_t cs) {
+  if (!c) return fail(SVT_EINVAL, "null cache");
+  if (!c->host_only) {
+    BuildParams bp{};
+    bp.n_streams = c->n_streams;
+    bp.S = std::max(1, c->S);
+    bp.ring_cap = c->ring_cap;
+    bp.sp_cap = std::max(1, c->sp_cap);
+    bp.max_pages = c->max_pages;
+    bp.scale = c->d_scale;
+    bp.ring = c->d_ring;
+    bp.special = c->d_special;
+    bp.indptr = c->d_indptr;
+    bp.indices = c->d_indices;
+    bp.lpl = c->d_lpl;
+    bp.err = c->d_err;
+    for (int i = 0; i < c->n_streams; ++i) {
+      const StreamState& s = c->st[i];
+      bp.s[i] = BuildStream{(int)s.scale.size(), s.ring_head, (int)s.window.size(),
+                            (int)s.special_pages.size(), page_valid_tokens_last(c, s)};
+    }
+    cudaError_t e = launch_build_table(bp, reinterpret_cast<cudaStream_t>(cs));
+    if (e != cudaSuccess) return cuda_fail(e, "table builder launch");
+  }
+  c->dirty = false;
+  c->plan_valid = false;
+  c->version += 1;
+  return SVT_OK;
+}
+
+int svt_read_device_page_table(svt_cache* c, int32_t* indptr, int32_t* indices,
+                               int32_t* last_page_len, int capacity, int* n_pages,
+                               svt_stream_t cs) {
+  if (!c) return fail(SVT_EINVAL, "null cache");
+  if (c->host_only) return fail(SVT_EINVAL, "host-only cache has no device table");
+  if (!indptr || !last_page_len) return fail(SVT_EINVAL, "null output");
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(cs);
+  cudaError_t e = cudaMemcpyAsync(indptr, c->d_indptr, sizeof(int) * (c->n_streams + 1),
+                                  cudaMemcpyDeviceToHost, s);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+  if (e != cudaSuccess) return cuda_fail(e, "read indptr");
+  int total = indptr[c->n_streams];
+  if (n_pages) *n_pages = total;
+  if (total < 0 || total > c->indices_cap) return fail(SVT_EDEVICE, "device indptr corrupt");
+  if (capacity < total) return fail(SVT_EINVAL, "capacity %d < %d entries", capacity, total);
+  if (total) {
+    if (!indices) return fail(SVT_EINVAL, "null indices");
+    e = cudaMemcpyAsync(indices, c->d_indices, sizeof(int) * total, cudaMemcpyDeviceToHost, s);
+  }
+  if (e == cudaSuccess)
+    e = cudaMemcpyAsync(last_page_len, c->d_lpl, sizeof(int) * c->n_streams,
+                        cudaMemcpyDeviceToHost, s);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+  if (e != cudaSuccess) return cuda_fail(e, "read device table");
+  return SVT_OK;
+}
+
+int svt_plan(svt_cache* c, const int32_t* qo_len, svt_stream_t) {
+  if (!c) return fail(SVT_EINVAL, "null cache");
+  if (!qo_len) return fail(SVT_EINVAL, "qo_len_per_stream is NULL");
+  if (c->dirty) return fail(SVT_ESTATE, "cache changed since build_visible_page_table");
+  const int P = c->P;
+  const int tpp = (P + kTileN - 1) / kTileN;
+  int rows = 0, page_off = 0;
+  AttnParams& a = c->attn;
+  SimtParams& m = c->simt;
+  a = AttnParams{};
+  m = SimtParams{};
+  svt_plan_info& info = c->info;
+  info = svt_plan_info{};
+  std::vector<int> tiles(c->n_streams, 0), qt(c->n_streams, 0);
+  for (int i = 0; i < c->n_streams; ++i) {
+    const StreamState& s = c->st[i];
+    const int np = n_visible_pages(s);
+    const int lpl = page_valid_tokens_last(c, s);
+    if (qo_len[i] < 0) return fail(SVT_EINVAL, "negative qo_len");
+    if (qo_len[i] > 0 && np == 0)
+      return fail(SVT_ESTATE, "stream %d has queries but no visible tokens", i);
+    if (c->rope_grid && qo_len[i] && qo_len[i] != c->ns + P)
+      return fail(SVT_EINVAL, "with RoPE each stream's query is one frame (%d rows)", c->ns + P);
+    StreamPlan& sp = a.s[i];
+    sp.q_off = rows;
+    sp.nq = qo_len[i];
+    sp.qtiles = (qo_len[i] + kTileM - 1) / kTileM;
+    sp.page_off = page_off;
+    sp.n_pages = np;
+    sp.lpl = lpl;
+    sp.tiles = np ? (np - 1) * tpp + (lpl + kTileN - 1) / kTileN : 0;
+    tiles[i] = sp.tiles;
+    qt[i] = sp.qtiles;
+    rows += qo_len[i];
+    page_off += np;
+    info.kv_tiles[i] = sp.tiles;
+    info.kv_tokens[i] = np ? (int64_t)(np - 1) * P + lpl : 0;
+    info.qo_len[i] = qo_len[i];
+  }
+  if (rows > c->max_qo) return fail(SVT_EINVAL, "total query rows %d > max_qo_len %d", rows, c->max_qo);
+  // Choose KV splits: candidate k scales every stream's chunk count with its tile count.
+  int max_tiles = 0;
+  for (int i = 0; i < c->n_streams; ++i)
+    if (qo_len[i]) max_tiles = std::max(max_tiles, tiles[i]);
+  const double tile_us = 4.0 * kTileM * kTileN * c->D / 5.5e6;   // ~50% of per-SM peak
+  const double item_us = 2.0;
+  std::vector<int> best(c->n_streams, 1);
+  double best_t = 1e300;
+  std::vector<double> cost;
+  for (int k = 1; k <= c->max_splits; ++k) {
+    std::vector<int> ch(c->n_streams, 1);
+    bool split = false;
+    cost.clear();
+    double merge_bytes = 0;
+    for (int i = 0; i < c->n_streams; ++i) {
+      if (!qo_len[i]) continue;
+      int cc = (int)std::ceil((double)k * tiles[i] / std::max(1, max_tiles));
+      cc = std::max(1, std::min({cc, c->max_splits, tiles[i]}));
+      ch[i] = cc;
+      if (cc > 1) {
+        split = true;
+        merge_bytes += (double)qo_len[i] * c->H * (c->D + 1) * 4.0 * (cc + 1);
+      }
+      for (int h = 0; h < c->H; ++h)
+        for (int cix = 0; cix < cc; ++cix)
+          for (int q = 0; q < qt[i]; ++q) {
+            int t0 = (int)((int64_t)cix * tiles[i] / cc), t1 = (int)((int64_t)(cix + 1) * tiles[i] / cc);
+            cost.push_back(item_us + (t1 - t0) * tile_us);
+          }
+    }
+    double t = simulate(cost, c->num_sms) + (split ? 4.0 + merge_bytes / 5.0e6 : 0.0);
+    if (t < best_t * 0.98) {
+      best_t = t;
+      best = ch;
+    }
+  }
+  int items = 0;
+  bool any_split = false;
+  for (int i = 0; i < c->n_streams; ++i) {
+    StreamPlan& sp = a.s[i];
+    sp.chunks = qo_len[i] ? best[i] : 0;
+    sp.item_off = items;
+    items += c->H * sp.qtiles * sp.chunks;
+    any_split |= sp.chunks > 1;
+    info.splits[i] = sp.chunks;
+  }
+  a.n_streams = c->n_streams;
+  a.total_items = items;
+  a.H = c->H;
+  a.D = c->D;
+  a.P = P;
+  a.max_pages = c->max_pages;
+  a.indices = c->d_indices;
+  a.scale_log2 = (float)(1.4426950408889634 / std::sqrt((double)c->D));
+  a.ws_o = c->d_ws_o;
+  a.ws_lse = c->d_ws_lse;
+  a.ws_rows = c->max_qo;
+  a.err = c->d_err;
+  info.num_items = items;
+  // fp32-FMA decomposition
+  const int rb = simt_rows_per_block(c->D);
+  int blocks = 0;
+  m.n_streams = c->n_streams;
+  for (int i = 0; i < c->n_streams; ++i) {
+    SimtStream& ss = m.s[i];
+    ss.q_off = a.s[i].q_off;
+    ss.nq = a.s[i].nq;
+    ss.rblocks = (a.s[i].nq + rb - 1) / rb;
+    ss.page_off = a.s[i].page_off;
+    ss.n_pages = a.s[i].n_pages;
+    ss.lpl = a.s[i].lpl;
+    ss.block_off = blocks;
+    blocks += ss.rblocks * c->H;
+  }
+  m.total_blocks = blocks;
+  m.H = c->H;
+  m.D = c->D;
+  m.P = P;
+  m.max_pages = c->max_pages;
+  m.indices = c->d_indices;
+  m.scale = (float)(1.0 / std::sqrt((double)c->D));
+  m.err = c->d_err;
+  c->total_rows = rows;
+  c->any_split = any_split;
+  c->plan_valid = true;
+  c->plan_version = c->version;
+  return SVT_OK;
+}
+
+int svt_get_plan_info(const svt_cache* c, svt_plan_info* out) {
+  if (!c || !out) return fail(SVT_EINVAL, "null argument");
+  if (!c->plan_valid) return fail(SVT_ESTATE, "no valid plan");
+  *out = c->info;
+  return SVT_OK;
+}
+
+int svt_run(svt_cache* c, int block, const void* q, void* out, float* lse, int force_fp32,
+            svt_stream_t cs) {
+  if (!c) return fail(SVT_EINVAL, "null cache");
+  if (c->host_only) return fail(SVT_EINVAL, "host-only cache cannot run kernels");
+  if (block < 0 || block >= c->L) return fail(SVT_EINVAL, "block %d out of range", block);
+  if (!c->plan_valid || c->plan_version != c->version || c->dirty)
+    return fail(SVT_ESTATE, "no valid plan for the current page table (build, then plan)");
+  if (c->total_rows == 0) return SVT_OK;
+  if (!q || !out) return fail(SVT_EINVAL, "q and out must be device pointers");
+  for (int i = 0; i < c->n_streams; ++i)
+    if (c->attn.s[i].nq && c->st[i].blocks_done <= block)
+      return fail(SVT_ESTATE, "stream %d: block %d has not appended the current frame", i, block);
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(cs);
+  const char* qsrc = static_cast<const char*>(q);
+  cudaError_t e;
+  if (c->rope_grid) {
+    RopeQParams rp{};
+    rp.q_in = qsrc;
+    rp.q_out = c->d_qrope;
+    rp.rows = c->total_rows;
+    rp.frame_rows = c->ns + c->P;
+    rp.ns = c->ns;
+    rp.H = c->H;
+    rp.D = c->D;
+    rp.elem = c->elem;
+    rp.rope_tab = c->d_rope_tab;
+    rp.rope_grid = c->rope_grid;
+    e = launch_rope_q(rp, c->dtype, s);
+    if (e != cudaSuccess) return cuda_fail(e, "rope_q launch");
+    qsrc = c->d_qrope;
+  }
+  const size_t block_bytes = (size_t)c->max_pages * 2 * c->P * c->H * c->D * c->elem;
+  if (force_fp32 || c->dtype == SVT_FP32) {
+    SimtParams m = c->simt;
+    m.pool_block = c->pool + (size_t)block * block_bytes;
+    m.q = qsrc;
+    m.out = static_cast<float*>(out);
+    m.lse = lse;
+    e = launch_attn_simt(m, c->dtype, s);
+    if (e != cudaSuccess) return cuda_fail(e, "fp32 attention launch");
+    return SVT_OK;
+  }
+  if (reinterpret_cast<uintptr_t>(qsrc) % 16) return fail(SVT_EINVAL, "q must be 16-byte aligned");
+  if (int r = encode_q_map(c, qsrc, c->total_rows)) return r;
+  AttnParams a = c->attn;
+  a.block_page_base = (int64_t)block * c->max_pages;
+  a.out = out;
+  a.lse = lse;
+  e = launch_attn_sm100(a, &c->tmap_q, &c->tmap_kv, c->dtype, s);
+  if (e != cudaSuccess) return cuda_fail(e, "attention launch");
+  if (c->any_split) {
+    e = launch_merge(a, c->dtype, s);
+    if (e != cudaSuccess) return cuda_fail(e, "merge launch");
+  }
+  return SVT_OK;
+}
+
+int svt_device_error(svt_cache* c, svt_stream_t cs) {
+  if (!c) return fail(SVT_EINVAL, "null cache");
+  if (c->host_only) return SVT_OK;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(cs);
+  unsigned h = 0;
+  cudaError_t e = cudaMemcpyAsync(&h, c->d_err, sizeof(h), cudaMemcpyDeviceToHost, s);
+  if (e == cudaSuccess) e = cudaMemsetAsync(c->d_err, 0, sizeof(unsigned), s);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+  if (e != cudaSuccess) return cuda_fail(e, "read device error word");
+  if (h)
+    return fail(SVT_EDEVICE, "device error 0x%x:%s%s%s", h, (h & kErrPageId) ? " page-id" : "",
+                (h & kErrWaitLimit) ? " wait-limit" : "", (h & kErrShape) ? " shape" : "");
+  return SVT_OK;
+}
+
+}  // extern "C"

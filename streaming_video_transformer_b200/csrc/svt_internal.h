@@ -1,0 +1,122 @@
+// Internal declarations shared by the host library (svt_cache.cu) and the
+// kernel files.  Not part of the C ABI.
+#pragma once
+
+#include <cstddef>
+#include <cstdint>
+#include <cuda_runtime.h>
+
+#include "../../include/svt.h"
+
+namespace svt {
+
+constexpr int kMaxSpecialSpan = 8;   // special pages one frame's specials can touch
+constexpr int kTileM = 128;          // query rows per tensor-core tile
+constexpr int kTileN = 128;          // KV tokens per tensor-core tile
+
+// Device error word bits (OR-ed by kernels, read by svt_device_error).
+enum : unsigned {
+  kErrPageId = 1u,      // a page id read from the device table is out of range
+  kErrWaitLimit = 2u,   // an mbarrier wait hit its iteration limit
+  kErrShape = 4u,       // a kernel found a shape it does not support
+};
+
+// ---------------------------------------------------------------- append
+struct AppendParams {
+  char* pool_block;          // pool region of this transformer block
+  const char* k;             // [Nq][H][D]
+  const char* v;
+  int ns, P, H, D, elem;     // elem = bytes per element
+  int patch_page;
+  int sp_off0;               // offset of the frame's first special token in sp_pages[0]
+  int n_sp;                  // special pages touched by this frame
+  int sp_pages[kMaxSpecialSpan];
+  // Block-0 update of the device page-table mirror (mirror_patch == nullptr otherwise).
+  int* mirror_patch;         // slot receiving patch_page
+  int* mirror_special;       // first slot receiving new special pages
+  int n_new_sp;
+  int new_sp[kMaxSpecialSpan];
+  const float2* rope_tab;    // [grid][D/4] (cos, sin), nullptr = no RoPE
+  int rope_grid;
+};
+cudaError_t launch_append(const AppendParams& p, int dtype, cudaStream_t s);
+
+// ------------------------------------------------------------- RoPE on Q
+struct RopeQParams {
+  const char* q_in;          // [rows][H][D]
+  char* q_out;
+  int rows, frame_rows, ns, H, D, elem;
+  const float2* rope_tab;
+  int rope_grid;
+};
+cudaError_t launch_rope_q(const RopeQParams& p, int dtype, cudaStream_t s);
+
+// -------------------------------------------------------- table builder
+struct BuildStream { int n_scale, ring_head, ring_len, n_special, lpl; };
+struct BuildParams {
+  int n_streams, S, ring_cap, sp_cap, max_pages;
+  const int* scale;          // [n_streams][S]
+  const int* ring;           // [n_streams][ring_cap]
+  const int* special;        // [n_streams][sp_cap]
+  int* indptr;               // [n_streams+1]
+  int* indices;
+  int* lpl;                  // [n_streams]
+  unsigned* err;
+  BuildStream s[SVT_MAX_STREAMS];
+};
+cudaError_t launch_build_table(const BuildParams& p, cudaStream_t s);
+
+// ------------------------------------------------------------ attention
+// Per-stream slice of one attention launch.
+struct StreamPlan {
+  int q_off;        // first query row of the stream in q / out
+  int nq;           // query rows
+  int qtiles;       // ceil(nq / kTileM)
+  int chunks;       // KV chunks (splits)
+  int page_off;     // first entry of the stream in the visible table
+  int n_pages;      // entries in the visible table
+  int lpl;          // valid tokens on the last page
+  int tiles;        // KV tiles: (n_pages-1)*ceil(P/kTileN) + ceil(lpl/kTileN)
+  int item_off;     // first work item of the stream
+};
+
+struct AttnParams {
+  int n_streams, total_items;
+  int H, D, P, max_pages;
+  int64_t block_page_base;   // block * max_pages (page coordinate of this block's page 0)
+  const int* indices;        // device visible table
+  float scale_log2;          // log2(e) / sqrt(D)
+  void* out;                 // [rows][H][D] cache dtype (used when chunks == 1)
+  float* lse;                // [rows][H] or nullptr
+  float* ws_o;               // [max_splits][ws_rows][H][D] fp32 partials
+  float* ws_lse;             // [max_splits][ws_rows][H]
+  int ws_rows;
+  unsigned* err;
+  StreamPlan s[SVT_MAX_STREAMS];
+};
+
+// Tensor-core (tcgen05 / TMEM) kernel; tensor maps are CUtensorMap (128 bytes each).
+cudaError_t launch_attn_sm100(const AttnParams& p, const void* tmap_q, const void* tmap_kv,
+                              int dtype, cudaStream_t s);
+
+// Combines split-KV partials into out / lse.
+cudaError_t launch_merge(const AttnParams& p, int dtype, cudaStream_t s);
+
+// fp32-FMA kernel (force_fp32 / fp32 pool).  Writes fp32 out and lse directly.
+struct SimtStream { int q_off, nq, rblocks, page_off, n_pages, lpl, block_off; };
+struct SimtParams {
+  int n_streams, total_blocks;
+  int H, D, P, max_pages;
+  const char* pool_block;
+  const int* indices;
+  const char* q;
+  float* out;
+  float* lse;
+  float scale;               // 1 / sqrt(D)
+  unsigned* err;
+  SimtStream s[SVT_MAX_STREAMS];
+};
+int simt_rows_per_block(int D);
+cudaError_t launch_attn_simt(const SimtParams& p, int dtype, cudaStream_t s);
+
+}  // namespace svt

@@ -1,0 +1,192 @@
+"""GPU parity at small sizes: the tiny stream, the hand-worked example,
+edge cases, and the invariants (page-id independence, rollback)."""
+import numpy as np
+import pytest
+import torch
+
+import golden_io
+from alloc_model import AllocModel
+from gpu_util import (FrameBank, assert_close, gather_visible, make_cache, max_pages_for,
+                      oracle_out, oracle_stream)
+from streaming_video_transformer_b200.inputs import WORKLOADS, small_workload
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _build():
+    from streaming_video_transformer_b200.build import build
+    build()
+
+
+def _step(cache, w, bank, t, blocks=(0,), stream=0, deferred=False):
+    q, k, v = bank.device(t)
+    if deferred:
+        cache.set_defer_eviction(True, stream)
+    for b in range(w.blocks):
+        cache.append_frame(b, k, v, stream=stream)
+    cache.evict_frames(stream)
+    cache.build_visible_page_table()
+    cache.plan([w.Nq])
+    return q
+
+
+def test_tiny_stream_every_frame():
+    """12 frames, one at a time: table, pool bytes and outputs every frame."""
+    w = WORKLOADS["tiny_stream"]
+    mp = max_pages_for(w, [w.frames])
+    c = make_cache(w, mp)
+    m = AllocModel(mp, w.P, w.ns, w.S, w.W)
+    bank = FrameBank(w, 0, 0)
+    st = oracle_stream(w)
+    counts = [int(x) for x in golden_io.visible_counts()["tiny"][1]]
+    for t in range(w.frames):
+        q = _step(c, w, bank, t)
+        m.append(0); m.evict(0)
+        q64, k64, v64 = bank.oracle(t)
+        st.append_frame(k64, v64)
+        # page tables: device == host == model
+        dip, dix, dlp = c.read_device_page_table()
+        hip, hix, hlp = c.get_page_table()
+        mip, mix, mlp = m.table()
+        assert list(dip) == list(hip) == mip and list(dix) == list(hix) == mix
+        assert list(dlp) == list(hlp) == mlp
+        # pool through the table == oracle visible K/V, bit for bit
+        gk, gv = gather_visible(c, 0, 0)
+        ok, ov = st.visible_kv()
+        assert gk.shape[0] == counts[t]
+        assert np.array_equal(gk, ok) and np.array_equal(gv, ov)
+        ref, ref_lse = oracle_out(st, q64)
+        lse = torch.empty((w.Nq, w.H), dtype=torch.float32, device="cuda")
+        out = c.run(0, q, lse=lse)
+        assert out.dtype == torch.bfloat16
+        assert_close(out, ref, what=f"t={t + 1}")
+        np.testing.assert_allclose(lse.cpu().numpy(), ref_lse, atol=2e-2)
+        out32 = c.run(0, q, force_fp32=True, lse=lse)
+        assert out32.dtype == torch.float32
+        assert_close(out32, ref, fp32=True, what=f"fp32 t={t + 1}")
+        np.testing.assert_allclose(lse.cpu().numpy(), ref_lse, atol=1e-5)
+    c.device_error()
+
+
+def test_hand_worked_example_on_gpu():
+    """The two-frame closed form, embedded in D=64 (zero features; q scaled
+    by 4 so that q.k/sqrt(64) equals the example's q.k/sqrt(4))."""
+    cases, _ = golden_io.two_frame_cases()
+    D = 64
+
+    def pad(rows):
+        x = torch.zeros((3, 1, D), dtype=torch.bfloat16)
+        for i, r in enumerate(rows):
+            x[i, 0, :4] = torch.tensor(r, dtype=torch.bfloat16)
+        return x.cuda()
+
+    q = pad([[8, 0, 0, 0], [0] * 4, [0] * 4])
+    f0 = (pad([[1, 0, 0, 0], [0] * 4, [0] * 4]), pad([[1, 0, 0, 0], [0, 1, 0, 0], [0, 0, 1, 0]]))
+    f1 = (pad([[0] * 4, [1, 0, 0, 0], [0] * 4]), pad([[0, 0, 0, 1], [1, 1, 0, 0], [0] * 4]))
+    for S, W, t, row, expected in cases:
+        c = make_cache(small_workload(P=2, ns=1, S=S, W=W, H=1, D=D), max_pages=12)
+        for k, v in (f0, f1)[:t]:
+            c.append_frame(0, k, v)
+            c.evict_frames()
+        c.build_visible_page_table()
+        c.plan([3])
+        out = c.run(0, q).float().cpu().numpy()
+        np.testing.assert_allclose(out[row, 0, :4], expected, atol=4e-3)
+        np.testing.assert_array_equal(out[row, 0, 4:], 0)
+        out32 = c.run(0, q, force_fp32=True).cpu().numpy()
+        np.testing.assert_allclose(out32[row, 0, :4], expected, atol=1e-6)
+
+
+EDGE = [
+    dict(P=16, ns=6, S=0, W=3, H=2, D=64, frames=7),              # no scale frames
+    dict(P=16, ns=6, S=2, W=0, H=2, D=64, frames=5),              # empty window
+    dict(P=8, ns=8, S=1, W=2, H=1, D=64, frames=6),               # last page always full
+    dict(P=200, ns=6, S=2, W=3, H=3, D=64, frames=6),             # page > 128 tokens: 2 tiles
+    dict(P=300, ns=6, S=1, W=2, H=2, D=128, frames=5, dtype="fp16"),
+    dict(P=16, ns=0, S=2, W=2, H=2, D=64, frames=5),              # no special tokens
+    dict(P=130, ns=6, S=3, W=4, H=4, D=64, frames=9),             # Nq 136: ragged q tile
+]
+
+
+@pytest.mark.parametrize("cfg", EDGE, ids=[str(i) for i in range(len(EDGE))])
+def test_edge_shapes(cfg):
+    w = small_workload(**cfg, R=cfg["frames"])
+    c = make_cache(w, max_pages_for(w, [w.frames]))
+    bank = FrameBank(w, 0, 0)
+    st = oracle_stream(w)
+    for t in range(w.frames):
+        q = _step(c, w, bank, t)
+        q64, k64, v64 = bank.oracle(t)
+        st.append_frame(k64, v64)
+        ref, _ = oracle_out(st, q64)
+        assert_close(c.run(0, q), ref, what=f"{cfg} t={t + 1}")
+        assert_close(c.run(0, q, force_fp32=True), ref, fp32=True, what=f"fp32 {cfg} t={t + 1}")
+        gk, gv = gather_visible(c, 0, 0)
+        ok, ov = st.visible_kv()
+        assert np.array_equal(gk, ok) and np.array_equal(gv, ov)
+    c.device_error()
+
+
+def test_page_ids_do_not_change_outputs():
+    w = small_workload(P=64, ns=6, S=2, W=3, H=2, D=64, frames=9, R=9)
+    mp = max_pages_for(w, [w.frames])
+    outs = []
+    for perm in (False, True):
+        c = make_cache(w, mp)
+        if perm:
+            rng = np.random.default_rng(3)
+            c.set_free_lists(rng.permutation(c.patch_pages),
+                             c.patch_pages + rng.permutation(mp - c.patch_pages))
+        bank = FrameBank(w, 0, 0, need_oracle=False)
+        for t in range(w.frames):
+            q = _step(c, w, bank, t)
+        outs.append((c.run(0, q).cpu(), c.run(0, q, force_fp32=True).cpu(), c.get_page_table()[1]))
+    assert not np.array_equal(outs[0][2], outs[1][2])           # different physical pages
+    assert torch.equal(outs[0][0], outs[1][0])                   # bit-identical outputs
+    assert torch.equal(outs[0][1], outs[1][1])
+
+
+def test_rollback_restores_outputs_bit_exactly():
+    w = small_workload(P=64, ns=6, S=2, W=3, H=2, D=64, frames=12, R=12, blocks=2)
+    c = make_cache(w, max_pages_for(w, [w.frames]))
+    bank = FrameBank(w, 0, 0, need_oracle=False)
+    for t in range(7):
+        q = _step(c, w, bank, t)
+    before = [c.run(b, q).cpu() for b in range(2)]
+    table = c.get_page_table()
+    q2 = _step(c, w, bank, 7, deferred=True)
+    during = c.run(0, q2).cpu()
+    c.rollback_last_frame()
+    c.set_defer_eviction(False)
+    c.build_visible_page_table()
+    c.plan([w.Nq])
+    after = [c.run(b, q).cpu() for b in range(2)]
+    for a, b in zip(before, after):
+        assert torch.equal(a, b)
+    for a, b in zip(table, c.get_page_table()):
+        assert np.array_equal(a, b)
+    assert during.shape == before[0].shape
+
+
+def test_multi_stream_with_idle_stream():
+    """Three streams in one pool, the middle one has no query this step."""
+    w = small_workload(P=32, ns=6, S=1, W=2, H=2, D=64, R=8)
+    ages = [3, 5, 8]
+    c = make_cache(w, max_pages_for(w, ages, num_streams=3), num_streams=3)
+    banks = [FrameBank(w, 0, s) for s in range(3)]
+    sts = [oracle_stream(w) for _ in range(3)]
+    for s, age in enumerate(ages):
+        for t in range(age):
+            q, k, v = banks[s].device(t)
+            c.append_frame(0, k, v, stream=s)
+            c.evict_frames(s)
+            sts[s].append_frame(*banks[s].oracle(t)[1:])
+    c.build_visible_page_table()
+    c.plan([w.Nq, 0, w.Nq])
+    qa = banks[0].device(ages[0] - 1)[0]
+    qc = banks[2].device(ages[2] - 1)[0]
+    out = c.run(0, torch.cat([qa, qc]))
+    for s, rows in ((0, slice(0, w.Nq)), (2, slice(w.Nq, 2 * w.Nq))):
+        ref, _ = oracle_out(sts[s], banks[s].oracle(ages[s] - 1)[0])
+        assert_close(out[rows], ref, what=f"stream {s}")
