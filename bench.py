@@ -1,0 +1,474 @@
+"""Benchmark: streamed frames/s of 24-block paged attention (and attention
+TFLOP/s against the B200 bf16 tensor peak).
+
+Workload (synthetic, shapes of a ViT-L/14 on 518 px frames): 24 transformer
+blocks, each with its own page-pool region; H=16, D=64, 1369 patches +
+6 special tokens per frame (page_size 1369), scale_frames 8, sliding window
+64, 2-D RoPE (37x37 grid, theta 100) on patch Q/K, bf16.  One step = one
+frame of the stream: for every block, append the frame's K/V (block 0 also
+evicts, builds the visible page table and plans), then run paged attention
+for the frame's 1375 queries.  The stream is pre-filled to the steady state
+(72 frames, appends only, untimed), then W warm-up frames, then K timed
+frames; the defaults (W=3, K=925) stream frames 0..999.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
+
+Prints one JSON line.  With N>1 (torchrun) every rank streams its own
+replica (no data exchange; weak scaling) and rank 0 prints.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "streamed frames/s (24-block paged attn) and attn TFLOP/s as % of bf16 peak"
+WORKLOAD = "vitl_stream24"
+# frames appended (no attention) before the warm-up steps
+PREFILL = {"vitl_stream24": 72, "vitl_step": 200}
+
+
+def _peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            p = json.load(f)
+        return p["bf16_tflops"], p["bf16_tflops_sustained"], p["hbm_gbs"], "measured"
+    except Exception:
+        return 1590.0, 1400.0, 6650.0, "fallback"
+
+
+def _config(w, extra=None):
+    desc = (f"{w.name}: {w.blocks} block(s), H={w.H}, D={w.D}, P=page={w.P}, {w.ns} special/frame, "
+            f"S={w.S}, W={w.W}, " + (f"2-D RoPE {w.rope_grid}x{w.rope_grid} theta={w.rope_theta:g}, "
+                                     if w.rope_grid else "no RoPE, ") + w.dtype)
+    cfg = {"workload": desc,
+           "blocks": w.blocks, "heads": w.H, "head_dim": w.D, "page_size": w.P,
+           "num_special": w.ns, "scale_frames": w.S, "sliding_window": w.W,
+           "parallelism": "replicas", "l2": "inputs larger than L2 (437 MB pool per block)"}
+    if extra:
+        cfg.update(extra)
+    return cfg
+
+
+def _visible(t, w):
+    """Visible tokens once t frames are in the stream (append + evict)."""
+    return min(t, w.S) * w.P + min(max(t - w.S, 0), w.W) * w.P + w.ns * t
+
+
+class ClockSampler:
+    """nvidia-smi clocks / throttle reasons sampled during the timed region."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index):
+        self.idx = device_index
+        self.proc = None
+        self.path = None
+
+    def __enter__(self):
+        try:
+            fd, self.path = tempfile.mkstemp(suffix=".csv")
+            os.close(fd)
+            self.out = open(self.path, "w")
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "200", "-i", str(self.idx)], stdout=self.out, stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+            self.out.close()
+
+    def summary(self):
+        if self.proc is None or not self.path:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unavailable"]}
+        rows = []
+        with open(self.path) as f:
+            for line in f:
+                parts = [x.strip() for x in line.split(",")]
+                if len(parts) >= 9:
+                    rows.append(parts)
+        os.unlink(self.path)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        mx = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({n for r in rows for n, v in zip(names, r[5:9]) if v.lower() == "active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(mx) if mx else None, "reasons": reasons,
+                "samples": len(rows),
+                "power_w_max": max((float(r[3]) for r in rows
+                                    if r[3].replace(".", "").isdigit()), default=None)}
+
+
+# ------------------------------------------------------------------ GPU arm
+def run_gpu(args, rank, world, local_rank):
+    import numpy as np
+    import torch
+    from dataclasses import replace
+
+    from streaming_video_transformer_b200.cache import PagedKVCache
+    from streaming_video_transformer_b200.inputs import WORKLOADS, frame_qkv
+
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    w = replace(WORKLOADS[args.workload], R=4)
+    L = w.blocks
+    prefill = PREFILL[args.workload]
+    e2e_steps = min(args.steps, max(8, args.steps // 4))
+    total_frames = prefill + args.warmup + args.steps + e2e_steps
+    max_pages = (w.S + w.W + 1) + math.ceil(total_frames * w.ns / w.P) + 2
+    cache = PagedKVCache(max_pages, w.P, w.H, w.D, w.W, w.S, num_blocks=L, num_special=w.ns,
+                         dtype=w.dtype, rope_grid=w.rope_grid, rope_theta=w.rope_theta,
+                         device=dev)
+    # R distinct frames per block: pinned host copies (end-to-end leg) and device copies.
+    host = [[[x.pin_memory() for x in frame_qkv(w, b, rank, i)] for i in range(w.R)]
+            for b in range(L)]
+    devin = [[[x.to(dev) for x in host[b][i]] for i in range(w.R)] for b in range(L)]
+    out = torch.empty((w.Nq, w.H, w.D), dtype=torch.bfloat16, device=dev)
+    stream = torch.cuda.current_stream()
+
+    t_frame = 0
+
+    def append_only(t):
+        for b in range(L):
+            q, k, v = devin[b][t % w.R]
+            cache.append_frame(b, k, v)
+        cache.evict_frames()
+
+    def step(t, inputs, ev=None, outs=None):
+        """One frame: append (+ evict/build/plan at block 0) and attention per block."""
+        for b in range(L):
+            q, k, v = inputs(b, t)
+            cache.append_frame(b, k, v)
+            if b == 0:
+                cache.evict_frames()
+                cache.build_visible_page_table()
+                cache.plan([w.Nq])
+            if ev is not None:
+                ev[0].record(stream)
+            cache.run(b, q, out=outs[b] if outs is not None else out)
+            if ev is not None:
+                ev[1].record(stream)
+                ev = None
+
+    dev_inputs = lambda b, t: devin[b][t % w.R]
+    for t in range(prefill):
+        append_only(t)
+    t_frame = prefill
+    for _ in range(args.warmup):
+        step(t_frame, dev_inputs)
+        t_frame += 1
+    info = cache.plan_info()
+    torch.cuda.synchronize()
+
+    def barrier():
+        if world > 1:
+            import torch.distributed as dist
+            dist.barrier()
+
+    # --- device-resident timed region ---------------------------------------
+    run_events = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+                  for _ in range(args.steps)]
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    first_timed = t_frame
+    barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(local_rank) as clk:
+        start.record(stream)
+        for i in range(args.steps):
+            step(t_frame, dev_inputs, ev=run_events[i])
+            t_frame += 1
+        end.record(stream)
+        torch.cuda.synchronize()
+    barrier()
+    elapsed_ms = start.elapsed_time(end)
+    run_ms = [a.elapsed_time(b) for a, b in run_events]        # block-0 run of each frame
+    cache.device_error()
+    clocks = clk.summary()
+    timed_frames = list(range(first_timed, t_frame))
+    flops_per_block = [4.0 * w.Nq * _visible(t + 1, w) * w.H * w.D for t in timed_frames]
+    total_flops = L * sum(flops_per_block)
+
+    # --- end-to-end: inputs copied from pinned host memory every frame -------
+    copy_stream = torch.cuda.Stream(device=dev)
+    stage = [[[torch.empty_like(x) for x in devin[b][0]] for b in range(L)] for _ in range(2)]
+    copied = [torch.cuda.Event() for _ in range(2)]
+    consumed = [torch.cuda.Event() for _ in range(2)]
+    res_host = torch.empty((w.Nq, w.H, w.D), dtype=torch.bfloat16).pin_memory()
+    e_start, e_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    h2d = 0
+
+    def enqueue_copy(i, t):
+        nonlocal h2d
+        with torch.cuda.stream(copy_stream):
+            copy_stream.wait_event(consumed[i % 2])
+            for b in range(L):
+                for dst, src in zip(stage[i % 2][b], host[b][t % w.R]):
+                    dst.copy_(src, non_blocking=True)
+                    h2d += src.numel() * src.element_size()
+            copied[i % 2].record(copy_stream)
+
+    for ev in consumed:
+        ev.record(stream)
+    barrier()
+    torch.cuda.synchronize()
+    t0 = t_frame
+    e_start.record(stream)
+    enqueue_copy(0, t0)
+    for i in range(e2e_steps):
+        if i + 1 < e2e_steps:
+            enqueue_copy(i + 1, t0 + i + 1)
+        stream.wait_event(copied[i % 2])
+        buf = stage[i % 2]
+        step(t0 + i, lambda b, t: buf[b])
+        consumed[i % 2].record(stream)
+        res_host.copy_(out, non_blocking=True)            # the frame's result (last block)
+    e_end.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    e2e_ms = e_start.elapsed_time(e_end)
+    h2d_per_step = h2d // e2e_steps
+    d2h_per_step = res_host.numel() * res_host.element_size()
+    e2e_flops = L * sum(4.0 * w.Nq * _visible(t0 + i + 1, w) * w.H * w.D for i in range(e2e_steps))
+
+    if world > 1:
+        import torch.distributed as dist
+        t = torch.tensor([elapsed_ms, e2e_ms], device=dev, dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        elapsed_ms, e2e_ms = float(t[0]), float(t[1])
+
+    # per block: append, [RoPE on Q], attention, [merge]; plus one table build per frame
+    kernels_per_step = L * (2 + (1 if w.rope_grid else 0)
+                            + (1 if max(info["splits"]) > 1 else 0)) + 1
+    return dict(elapsed_ms=elapsed_ms, run_ms=run_ms, flops_per_block=flops_per_block,
+                total_flops=total_flops, clocks=clocks, info=info, w=w,
+                e2e_ms=e2e_ms, e2e_steps=e2e_steps, e2e_flops=e2e_flops,
+                h2d_per_step=h2d_per_step, d2h_per_step=d2h_per_step,
+                kernels_per_step=kernels_per_step, first_timed=first_timed, last_timed=t_frame)
+
+
+# ------------------------------------------------------------- CPU oracle
+def oracle_block_frame_seconds(w, t_frames, rows=None, heads=None):
+    """Times the oracle on one block at a cache holding t_frames frames."""
+    import numpy as np
+    import torch
+
+    from oracle import FrameStream, attend, rope2d
+    from streaming_video_transformer_b200.inputs import frame_qkv
+
+    st = FrameStream(w.P, w.ns, w.S, w.W)
+    data = []
+    for i in range(w.R):
+        q, k, v = frame_qkv(w, 0, 0, i)
+        qr = torch.from_numpy(rope2d(q, w.ns, w.rope_grid, w.rope_theta)).to(q.dtype)
+        kr = torch.from_numpy(rope2d(k, w.ns, w.rope_grid, w.rope_theta)).to(k.dtype)
+        data.append(tuple(x.double().numpy() for x in (qr, kr, v)))
+    for t in range(t_frames):
+        st.append_frame(data[t % w.R][1], data[t % w.R][2])
+    q = data[(t_frames - 1) % w.R][0]
+    if rows is not None:
+        q = q[rows]
+    t0 = time.perf_counter()
+    k, v = st.visible_kv()
+    if heads is not None:
+        k, v, q = k[:, heads], v[:, heads], q[:, heads]
+    attend(q, k, v)
+    return time.perf_counter() - t0
+
+
+def cpu_threads():
+    try:
+        return len(os.sched_getaffinity(0))
+    except Exception:
+        return os.cpu_count() or 1
+
+
+def run_reference(args):
+    """The CPU oracle as it stands, on the same workload: each step streams
+    one frame into the oracle's cache and computes attention for a sample of
+    the frame's query rows of one head of one block."""
+    import numpy as np
+    import torch
+    from dataclasses import replace
+
+    from oracle import FrameStream, attend, rope2d
+    from streaming_video_transformer_b200.inputs import WORKLOADS, frame_qkv
+
+    w = replace(WORKLOADS[WORKLOAD], R=4)
+    data = []
+    for i in range(w.R):
+        q, k, v = frame_qkv(w, 0, 0, i)
+        qr = torch.from_numpy(rope2d(q, w.ns, w.rope_grid, w.rope_theta)).to(q.dtype)
+        kr = torch.from_numpy(rope2d(k, w.ns, w.rope_grid, w.rope_theta)).to(k.dtype)
+        data.append(tuple(x.double().numpy() for x in (qr, kr, v)))
+    st = FrameStream(w.P, w.ns, w.S, w.W)
+    prefill = w.S + w.W
+    for t in range(prefill):
+        st.append_frame(data[t % w.R][1], data[t % w.R][2])
+    budget_s = float(os.environ.get("SVT_REFERENCE_BUDGET_S", "150"))
+    n_steps = args.warmup + args.steps
+    rows_n = 64
+    rng = np.random.default_rng(0)
+    per_frame = []
+    t_frame = prefill
+    for i in range(n_steps):
+        t_frame += 1
+        q, k, v = data[(t_frame - 1) % w.R]
+        st.append_frame(k, v)
+        h = i % w.H
+        t0 = time.perf_counter()
+        kv, vv = st.visible_kv()
+        kh, vh = kv[:, h:h + 1], vv[:, h:h + 1]
+        t1 = time.perf_counter()
+        rows = np.sort(rng.choice(w.Nq, size=rows_n, replace=False))
+        attend(q[rows][:, h:h + 1], kh, vh)
+        t2 = time.perf_counter()
+        # one frame = 24 blocks x (gather all heads once + attention of all rows x heads)
+        frame_s = w.blocks * ((t1 - t0) + w.H * (t2 - t1) * (w.Nq / rows_n))
+        if i >= args.warmup:
+            per_frame.append(frame_s)
+        if i == 0:   # size the row sample so the whole run stays within the budget
+            per_step = max(1e-3, budget_s / max(1, n_steps))
+            rows_n = int(max(1, min(w.Nq, rows_n * max(0.05, (per_step - (t1 - t0)) /
+                                                       max(t2 - t1, 1e-4)))))
+    mean_frame = sum(per_frame) / max(1, len(per_frame))
+    fps = 1.0 / mean_frame
+    flops = w.blocks * 4.0 * w.Nq * _visible(t_frame, w) * w.H * w.D
+    return {
+        "impl": "reference", "metric": METRIC, "value": fps, "unit": "frames/s",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": 1e3 * mean_frame, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": _config(w, {"frames": f"{prefill}..{t_frame - 1}"}),
+        "tflops": flops / mean_frame / 1e12,
+        "cpu_baseline": {"value": fps, "unit": "frames/s", "cores": cpu_threads(),
+                         "kind": "oracle",
+                         "sample": f"per step: stream one frame into the oracle, gather the "
+                                   f"visible K/V, attention for {rows_n} sampled rows of one head "
+                                   f"of one block; frame time = 24 x (gather + 16 heads x "
+                                   f"1375/{rows_n} x sampled attention)"},
+        "e2e": {"value": fps, "unit": "frames/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+
+
+# ---------------------------------------------------------------------- main
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=925)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="svt", choices=["svt", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--workload", default=WORKLOAD, choices=sorted(PREFILL),
+                    help="vitl_step (1 block, no RoPE) is the small case used for profiling")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+
+    if args.impl == "reference":
+        if rank == 0:
+            print(json.dumps(run_reference(args)), flush=True)
+        return
+
+    if world > 1:
+        import datetime
+        import torch
+        import torch.distributed as dist
+        torch.cuda.set_device(local_rank)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=600),
+                                device_id=torch.device("cuda", local_rank))
+    from streaming_video_transformer_b200.build import build
+    if rank == 0:
+        build()
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+    r = run_gpu(args, rank, world, local_rank)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+    if rank != 0:
+        return
+    w = r["w"]
+    burst, sustained, hbm, peak_kind = _peaks()
+    fps = world * args.steps / (r["elapsed_ms"] / 1e3)
+    tflops = r["total_flops"] / (r["elapsed_ms"] / 1e3) / 1e12
+    run_avg_ms = sum(r["run_ms"]) / len(r["run_ms"])
+    run_flops = sum(r["flops_per_block"]) / len(r["flops_per_block"])
+    achieved = run_flops / (run_avg_ms / 1e3) / 1e12
+    traffic = None
+    try:
+        with open(os.path.join(ROOT, "profiles", "attn_traffic.json")) as f:
+            tr = json.load(f)
+            traffic = tr.get("dram_bytes_per_launch")
+    except Exception:
+        pass
+    cpu = None
+    if not args.no_cpu_baseline and world == 1:
+        try:
+            secs = oracle_block_frame_seconds(w, r["last_timed"])
+            cpu = {"value": 1.0 / (w.blocks * secs), "unit": "frames/s", "cores": cpu_threads(),
+                   "kind": "oracle",
+                   "sample": f"one of 24 blocks at frame t={r['last_timed']} (all 1375 query rows, "
+                             f"16 heads, {_visible(r['last_timed'], w)} visible tokens); "
+                             f"{secs:.1f} s x 24 blocks per frame"}
+        except Exception as exc:  # the CPU leg never blocks the GPU number
+            cpu = {"value": None, "unit": "frames/s", "cores": cpu_threads(), "kind": "oracle",
+                   "sample": f"failed: {exc!r}"}
+    e2e_fps = world * r["e2e_steps"] / (r["e2e_ms"] / 1e3)
+    line = {
+        "metric": METRIC, "value": fps, "unit": "frames/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": r["elapsed_ms"] / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic",
+        "config": _config(w, {"frames": f"pre-filled 0..{w.S + w.W - 1}, warm-up to "
+                                        f"{r['first_timed'] - 1}, timed {r['first_timed']}.."
+                                        f"{r['last_timed'] - 1}",
+                              "splits": r["info"]["splits"][0],
+                              "work_items": r["info"]["num_items"]}),
+        "tflops": tflops,
+        "tflops_frac_of_peak": {"burst": tflops / burst, "sustained": tflops / sustained,
+                                "peak_kind": peak_kind},
+        "roofline": {"bound": "tensor", "achieved": achieved, "peak": sustained,
+                     "unit": "TFLOP/s", "frac": achieved / sustained, "traffic": traffic,
+                     "kernel": "svt_run (RoPE on Q + tcgen05 attention + split merge), block 0 "
+                               "of every timed frame, CUDA events on the launch stream",
+                     "peak_kind": f"bf16 sustained ({peak_kind})",
+                     "frac_of_burst": achieved / burst},
+        "cpu_baseline": cpu,
+        "e2e": {"value": e2e_fps, "unit": "frames/s", "h2d_bytes_per_step": r["h2d_per_step"],
+                "d2h_bytes_per_step": r["d2h_per_step"], "steps": r["e2e_steps"],
+                "note": "inputs of all 24 blocks copied from pinned host memory each frame on a "
+                        "copy stream (double-buffered), last block's output read back"},
+        "gpu_launches": r["kernels_per_step"] * args.steps,
+        "clocks": r["clocks"],
+    }
+    print(json.dumps(line), flush=True)
+
+
+if __name__ == "__main__":
+    main()

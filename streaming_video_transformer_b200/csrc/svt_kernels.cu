@@ -230,14 +230,18 @@ __global__ void __launch_bounds__(kSimtThreads) attn_simt_kernel(SimtParams p) {
   const int r = rblock * RB + threadIdx.x / TPR;
   const bool active = r < S.nq;
   const size_t HD = (size_t)p.H * D;
-  float q[32], o[32];
+  // o and l are accumulated per tile (32 terms) and the tile sums are added
+  // into the running totals with Kahan compensation (oc, lc), so that streams
+  // of 10^5 keys keep fp32 rounding at the level of a few ulps.
+  float q[32], o[32], oc[32];
   const T* qrow = reinterpret_cast<const T*>(p.q) + (size_t)(S.q_off + (active ? r : 0)) * HD + h * D + part * 32;
 #pragma unroll
   for (int i = 0; i < 32; ++i) {
     q[i] = active ? to_f(qrow[i]) : 0.f;
     o[i] = 0.f;
+    oc[i] = 0.f;
   }
-  float m = -INFINITY, l = 0.f;
+  float m = -INFINITY, l = 0.f, lc = 0.f;
   const T* pool = reinterpret_cast<const T*>(p.pool_block);
   for (int pp = 0; pp < S.n_pages; ++pp) {
     int page = p.indices[S.page_off + pp];
@@ -264,7 +268,7 @@ __global__ void __launch_bounds__(kSimtThreads) attn_simt_kernel(SimtParams p) {
       __syncthreads();
       float s[kSimtKT];
       float tmax = -INFINITY;
-#pragma unroll 4
+#pragma unroll
       for (int j = 0; j < kSimtKT; ++j) {
         float acc = 0.f;
 #pragma unroll
@@ -276,16 +280,31 @@ __global__ void __launch_bounds__(kSimtThreads) attn_simt_kernel(SimtParams p) {
       }
       const float mnew = fmaxf(m, tmax);
       const float alpha = expf(m - mnew);   // m = -inf on the first tile -> 0
-      l *= alpha;
-#pragma unroll
-      for (int i = 0; i < 32; ++i) o[i] *= alpha;
       m = mnew;
-#pragma unroll 4
+      float ot[32], lt = 0.f;
+#pragma unroll
+      for (int i = 0; i < 32; ++i) ot[i] = 0.f;
+#pragma unroll
       for (int j = 0; j < kSimtKT; ++j) {
         const float pj = expf(s[j] - m);
-        l += pj;
+        lt += pj;
 #pragma unroll
-        for (int i = 0; i < 32; ++i) o[i] = fmaf(pj, vs[j][part][i], o[i]);
+        for (int i = 0; i < 32; ++i) ot[i] = fmaf(pj, vs[j][part][i], ot[i]);
+      }
+      {
+        const float lr = __fmul_rn(l, alpha), lcr = __fmul_rn(lc, alpha);
+        const float y = __fsub_rn(lt, lcr);
+        const float tt = __fadd_rn(lr, y);
+        lc = __fsub_rn(__fsub_rn(tt, lr), y);
+        l = tt;
+      }
+#pragma unroll
+      for (int i = 0; i < 32; ++i) {
+        const float orr = __fmul_rn(o[i], alpha), ocr = __fmul_rn(oc[i], alpha);
+        const float y = __fsub_rn(ot[i], ocr);
+        const float tt = __fadd_rn(orr, y);
+        oc[i] = __fsub_rn(__fsub_rn(tt, orr), y);
+        o[i] = tt;
       }
     }
   }

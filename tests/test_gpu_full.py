@@ -103,8 +103,11 @@ def test_vitl_stream24_blocks_0_and_23():
     gk, gv = gather_visible(c, 23, 0)
     ok, ov = sts[23].visible_kv()
     assert np.array_equal(gv, ov)
+    # fp32 rotation vs float64 rotation, each rounded once to bf16: within one
+    # bf16 step of the value plus the fp32 arithmetic error of the rotation
+    # (a few 2^-24 of the input's magnitude, which dominates after cancellation).
     diff = np.abs(gk - ok)
-    assert np.max(diff / np.maximum(np.abs(ok), 1e-30)) <= 2.0 ** -8
+    assert np.all(diff <= 2.0 ** -8 * np.abs(ok) + 4e-6)
     assert np.mean(diff > 0) < 1e-3
     c.device_error()
 
