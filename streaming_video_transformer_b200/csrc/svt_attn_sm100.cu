@@ -10,21 +10,25 @@
 // table, each full except the last (last_page_len valid tokens) -- with no
 // causal mask, read straight from the page pool.
 //
-// Work item = (stream, head, 128-row query tile, KV chunk).  One CTA per item:
-//   warp 4      TMA producer: Q tile once, then K and V tiles of 128 tokens,
-//               gathered page by page through the visible table (a page of
-//               page_size tokens is ceil(page_size/128) tiles; rows past the
-//               page end are zero-filled by TMA and masked).
-//   warp 5      MMA issuer (one thread) and TMEM owner:
-//                 S_j = Q K_j^T      (SS MMA, fp32 into TMEM, double buffered)
-//                 O  += P_j V_j      (TS MMA: P_j read from TMEM, V_j from smem)
-//   warps 0-3   softmax: thread r owns query row r = TMEM lane r; reads S_j,
-//               online softmax in the log2 domain with a lazy rescale of O
-//               (only when the running max grows by more than 2^8), writes
-//               P_j as 16-bit pairs over the first half of S_j's columns,
-//               then the epilogue (O / l, LSE).
-// S_{j+1} is computed while the softmax works on S_j.  Split-KV chunks write
-// fp32 partials and LSE; a merge kernel combines them.
+// Work item = (stream, head, pair of 128-row query tiles, KV chunk); one CTA
+// per item, 320 threads:
+//   warp 8      TMA producer: both Q tiles once, then K and V tiles of 128
+//               tokens gathered page by page through the visible table (a
+//               page is ceil(page_size/128) tiles; rows past the page end are
+//               zero-filled by TMA and masked).
+//   warp 9      MMA issuer (one thread) and TMEM owner.  Per KV tile j:
+//                 S0_j = Q0 K_j^T, S1_j = Q1 K_j^T       (SS MMA into TMEM)
+//                 O0 += P0_j V_j,  O1 += P1_j V_j        (TS MMA, P from TMEM)
+//               in the order S0_0 S1_0 | PV0_0 S0_1 PV1_0 S1_1 | PV0_1 ...
+//   warps 0-3   softmax of query tile 0, warps 4-7 of query tile 1: thread r
+//               owns row r (TMEM lane r), reads S, keeps the running max and
+//               sum in the log2 domain, rescales O lazily (only when the max
+//               grows by more than 2^8), writes P as 16-bit pairs over the
+//               first half of S's columns; then the epilogue (O / l, LSE).
+// The two softmax warpgroups ping-pong: one works on its S while the tensor
+// cores run the other tile's P.V and next S.  K/V tiles are loaded once for
+// both query tiles.  Split-KV chunks write fp32 partials and LSE; a merge
+// kernel combines them.
 
 #include <cuda.h>
 #include <cuda_bf16.h>
@@ -33,12 +37,16 @@
 #include "sm100_primitives.cuh"
 #include "svt_internal.h"
 
+#ifndef SVT_EXP_MODE
+#define SVT_EXP_MODE 0   // 0: fp32 MUFU exp2; 1: packed f16x2 MUFU exp2 (two per instruction)
+#endif
+
 namespace svt {
 namespace {
 
 using namespace sm100;
 
-constexpr int kThreads = 192;
+constexpr int kThreads = 320;
 constexpr int kTmemCols = 512;
 constexpr uint64_t kWaitLimitNs = 2000000000ull;   // 2 s
 constexpr float kRescaleThreshold = 8.0f;          // log2 units
@@ -46,23 +54,24 @@ constexpr float kRescaleThreshold = 8.0f;          // log2 units
 template <int D>
 struct Cfg {
   static constexpr int kRegions = D / 64;                      // 64-feature swizzle columns
-  static constexpr uint32_t kTileBytes = kTileN * D * 2;       // one K or V (or Q) tile
+  static constexpr uint32_t kTileBytes = kTileN * D * 2;       // one K, V or Q tile
   static constexpr uint32_t kRegionBytes = kTileN * 128;       // 128 rows x 128 bytes
   static constexpr int kStages = D == 64 ? 4 : 2;
-  static constexpr uint32_t kQOff = 0;
-  static constexpr uint32_t kKOff = kTileM * D * 2;
+  static constexpr uint32_t kQOff = 0;                          // two Q tiles
+  static constexpr uint32_t kKOff = 2 * kTileBytes;
   static constexpr uint32_t kVOff = kKOff + kStages * kTileBytes;
   static constexpr uint32_t kBarOff = kVOff + kStages * kTileBytes;
-  // barriers: q_full, k_full[S], k_empty[S], v_full[S], v_empty[S], s_full[2], p_full[2],
-  // o_done[2] (PV_j commits to o_done[j&1]), drain ; then tmem base word and abort flag
+  // q_full, k_full[S], k_empty[S], v_full[S], v_empty[S], s_full[2], p_full[2], o_done[2], drain
   static constexpr int kNumBars = 1 + 4 * kStages + 2 + 2 + 2 + 1;
   static constexpr uint32_t kMiscOff = kBarOff + kNumBars * 8;
   static constexpr uint32_t kSmemBytes = kMiscOff + 16 + 1024;   // + alignment slack
-  static constexpr uint32_t kTmemS0 = 0, kTmemS1 = 128, kTmemO = 256;
+  static constexpr uint32_t kTmemS = 0;        // S of tile x at column 128 x
+  static constexpr uint32_t kTmemO = 256;      // O of tile x at column 256 + D x
 };
 
 struct Item {
-  int st, head, qtile, chunk, t_begin, n_tiles;
+  int st, head, qpair, chunk, t_begin, n_tiles;
+  bool two;   // the pair's second query tile holds rows of this stream
 };
 
 __device__ __forceinline__ Item decode_item(const AttnParams& p) {
@@ -70,12 +79,14 @@ __device__ __forceinline__ Item decode_item(const AttnParams& p) {
   int st = 0;
   while (st + 1 < p.n_streams && (int)blockIdx.x >= p.s[st + 1].item_off) ++st;
   const StreamPlan& sp = p.s[st];
+  const int qpairs = (sp.qtiles + 1) / 2;
   const int local = blockIdx.x - sp.item_off;
   it.st = st;
-  it.qtile = local % sp.qtiles;
-  const int rest = local / sp.qtiles;
+  it.qpair = local % qpairs;
+  const int rest = local / qpairs;
   it.chunk = rest % sp.chunks;
   it.head = rest / sp.chunks;
+  it.two = 2 * it.qpair + 1 < sp.qtiles;
   const int t0 = (int)((int64_t)it.chunk * sp.tiles / sp.chunks);
   const int t1 = (int)((int64_t)(it.chunk + 1) * sp.tiles / sp.chunks);
   it.t_begin = t0;
@@ -101,8 +112,19 @@ __device__ __forceinline__ void tile_coords(const StreamPlan& sp, int P, int g, 
   valid = min(kTileN, page_tokens - t * kTileN);
 }
 
+template <bool BF16>
+__device__ __forceinline__ uint32_t pack2(float lo, float hi) {
+  if constexpr (BF16) {
+    __nv_bfloat162 h2 = __floats2bfloat162_rn(lo, hi);
+    return *reinterpret_cast<uint32_t*>(&h2);
+  } else {
+    __half2 h2 = __floats2half2_rn(lo, hi);
+    return *reinterpret_cast<uint32_t*>(&h2);
+  }
+}
+
 template <int D, bool BF16>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __maxnreg__(192)
     attn_sm100_kernel(const __grid_constant__ CUtensorMap tmap_q,
                       const __grid_constant__ CUtensorMap tmap_kv,
                       const __grid_constant__ AttnParams p) {
@@ -116,14 +138,14 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t sK = base + C::kKOff;
   const uint32_t sV = base + C::kVOff;
   const uint32_t bars = base + C::kBarOff;
-  auto q_full = [&]() { return bars; };
+  const uint32_t q_full = bars;
   auto k_full = [&](int s) { return bars + 8u * (1 + s); };
   auto k_empty = [&](int s) { return bars + 8u * (1 + C::kStages + s); };
   auto v_full = [&](int s) { return bars + 8u * (1 + 2 * C::kStages + s); };
   auto v_empty = [&](int s) { return bars + 8u * (1 + 3 * C::kStages + s); };
-  auto s_full = [&](int b) { return bars + 8u * (1 + 4 * C::kStages + b); };
-  auto p_full = [&](int b) { return bars + 8u * (3 + 4 * C::kStages + b); };
-  auto o_done = [&](int b) { return bars + 8u * (5 + 4 * C::kStages + b); };
+  auto s_full = [&](int x) { return bars + 8u * (1 + 4 * C::kStages + x); };
+  auto p_full = [&](int x) { return bars + 8u * (3 + 4 * C::kStages + x); };
+  auto o_done = [&](int x) { return bars + 8u * (5 + 4 * C::kStages + x); };
   const uint32_t drain = bars + 8u * (7 + 4 * C::kStages);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(gbase + C::kMiscOff);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(gbase + C::kMiscOff + 4);
@@ -136,24 +158,23 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (threadIdx.x == 0) {
     *abort_flag = 0;
-    mbar_init(q_full(), 1);
+    mbar_init(q_full, 1);
     for (int s = 0; s < C::kStages; ++s) {
       mbar_init(k_full(s), 1);
       mbar_init(k_empty(s), 1);
       mbar_init(v_full(s), 1);
       mbar_init(v_empty(s), 1);
     }
-    for (int b = 0; b < 2; ++b) {
-      mbar_init(s_full(b), 1);
-      mbar_init(p_full(b), 128);
+    for (int x = 0; x < 2; ++x) {
+      mbar_init(s_full(x), 1);
+      mbar_init(p_full(x), 128);
+      mbar_init(o_done(x), 1);
     }
-    mbar_init(o_done(0), 1);
-    mbar_init(o_done(1), 1);
     mbar_init(drain, 1);
     fence_barrier_init();
     fence_proxy_async_shared();
   }
-  if (warp == 5) {
+  if (warp == 9) {
     tmem_alloc(smem_addr(tmem_slot), kTmemCols);
     tmem_relinquish();
   }
@@ -167,15 +188,17 @@ __global__ void __launch_bounds__(kThreads, 1)
     atomicOr(p.err, kErrWaitLimit);
   };
 
-  if (warp == 4) {
+  if (warp == 8) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
       tma_prefetch_desc(&tmap_q);
       tma_prefetch_desc(&tmap_kv);
-      mbar_arrive_expect_tx(q_full(), kTileM * D * 2);
-      for (int r = 0; r < C::kRegions; ++r)
-        tma_load_3d(sQ + r * C::kRegionBytes, &tmap_q, q_full(), r * 64, it.head,
-                    sp.q_off + it.qtile * kTileM);
+      const int q_row0 = sp.q_off + 2 * it.qpair * kTileM;
+      mbar_arrive_expect_tx(q_full, (it.two ? 2 : 1) * C::kTileBytes);
+      for (int x = 0; x < (it.two ? 2 : 1); ++x)
+        for (int r = 0; r < C::kRegions; ++r)
+          tma_load_3d(sQ + x * C::kTileBytes + r * C::kRegionBytes, &tmap_q, q_full, r * 64,
+                      it.head, q_row0 + x * kTileM);
       int issued = 0;
       for (int j = 0; j < n; ++j) {
         int page_pos, t, valid;
@@ -193,16 +216,16 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int r = 0; r < C::kRegions; ++r)
           tma_load_5d(sK + s * C::kTileBytes + r * C::kRegionBytes, &tmap_kv, k_full(s), r * 64,
                       it.head, t * kTileN, 0, c4);
-        if (!mbar_wait(v_empty(s), ph ^ 1, abort_flag, kWaitLimitNs)) { fail(); issued = j + 1; break; }
+        issued = j + 1;
+        if (!mbar_wait(v_empty(s), ph ^ 1, abort_flag, kWaitLimitNs)) { fail(); break; }
         mbar_arrive_expect_tx(v_full(s), C::kTileBytes);
         for (int r = 0; r < C::kRegions; ++r)
           tma_load_5d(sV + s * C::kTileBytes + r * C::kRegionBytes, &tmap_kv, v_full(s), r * 64,
                       it.head, t * kTileN, 1, c4);
-        issued = j + 1;
       }
       if (*abort_flag) {
         // Let the copies already in flight land before the CTA exits.
-        mbar_wait(q_full(), 0, nullptr, kWaitLimitNs);
+        mbar_wait(q_full, 0, nullptr, kWaitLimitNs);
         for (int j = max(0, issued - C::kStages); j < issued; ++j) {
           const int s = j % C::kStages;
           const uint32_t ph = (j / C::kStages) & 1;
@@ -211,135 +234,178 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
     }
-  } else if (warp == 5) {
+  } else if (warp == 9) {
     // ---------------------------------------------------------- MMA issuer
     if (lane == 0) {
       constexpr uint32_t idS = idesc_f16(kTileM, kTileN, BF16, false);
       constexpr uint32_t idO = idesc_f16(kTileM, D, BF16, true);
-      bool ok = mbar_wait(q_full(), 0, abort_flag, kWaitLimitNs);
-      if (!ok) fail();
+      const int nx = it.two ? 2 : 1;
+      bool ok = mbar_wait(q_full, 0, abort_flag, kWaitLimitNs);
       tc_fence_after();
-      auto issue_s = [&](int j) -> bool {
-        const int s = j % C::kStages;
-        if (!mbar_wait(k_full(s), (j / C::kStages) & 1, abort_flag, kWaitLimitNs)) return false;
-        tc_fence_after();
-        const uint32_t d = tmem + ((j & 1) ? C::kTmemS1 : C::kTmemS0);
-        const uint32_t kb = sK + s * C::kTileBytes;
+      // S_x = Q_x K_j^T into tile x's S columns.
+      auto issue_s = [&](int x, int j) {
+        const uint32_t kb = sK + (j % C::kStages) * C::kTileBytes;
+        const uint32_t qb = sQ + x * C::kTileBytes;
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t off = (kk / 4) * C::kRegionBytes + (kk % 4) * 32;
-          mma_ss(d, desc_sw128(sQ + off, 16, 1024), desc_sw128(kb + off, 16, 1024), idS,
-                 kk > 0 ? 1u : 0u);
+          mma_ss(tmem + C::kTmemS + 128 * x, desc_sw128(qb + off, 16, 1024),
+                 desc_sw128(kb + off, 16, 1024), idS, kk > 0 ? 1u : 0u);
         }
-        mma_commit(k_empty(s));
-        mma_commit(s_full(j & 1));
-        return true;
+        mma_commit(s_full(x));
       };
-      if (ok && n > 0) ok = issue_s(0);
-      for (int j = 0; ok && j < n; ++j) {
-        if (j + 1 < n && !(ok = issue_s(j + 1))) break;
-        if (!(ok = mbar_wait(p_full(j & 1), (j >> 1) & 1, abort_flag, kWaitLimitNs))) break;
-        tc_fence_after();
-        const int s = j % C::kStages;
-        const uint32_t vb = sV + s * C::kTileBytes;
-        const uint32_t a = tmem + ((j & 1) ? C::kTmemS1 : C::kTmemS0);
+      // O_x += P_x V_j with P_x read from tile x's S columns.
+      auto issue_pv = [&](int x, int j) {
+        const uint32_t vb = sV + (j % C::kStages) * C::kTileBytes;
+        const uint32_t a = tmem + C::kTmemS + 128 * x;
 #pragma unroll
         for (int kk = 0; kk < kTileN / 16; ++kk)
-          mma_ts(tmem + C::kTmemO, a + kk * 8, desc_sw128(vb + kk * 2048, C::kRegionBytes, 1024),
-                 idO, (j > 0 || kk > 0) ? 1u : 0u);
-        mma_commit(v_empty(s));
-        mma_commit(o_done(j & 1));
+          mma_ts(tmem + C::kTmemO + D * x, a + kk * 8,
+                 desc_sw128(vb + kk * 2048, C::kRegionBytes, 1024), idO,
+                 (j > 0 || kk > 0) ? 1u : 0u);
+      };
+      if (ok && n > 0) {
+        ok = mbar_wait(k_full(0), 0, abort_flag, kWaitLimitNs);
+        if (ok) {
+          tc_fence_after();
+          for (int x = 0; x < nx; ++x) issue_s(x, 0);
+          mma_commit(k_empty(0));
+        }
+      }
+      for (int j = 0; ok && j < n; ++j) {
+        const int s = j % C::kStages;
+        const int s1 = (j + 1) % C::kStages;
+        const bool more = j + 1 < n;
+        for (int x = 0; x < nx && ok; ++x) {
+          if (!(ok = mbar_wait(p_full(x), j & 1, abort_flag, kWaitLimitNs))) break;
+          if (x == 0 && !(ok = mbar_wait(v_full(s), (j / C::kStages) & 1, abort_flag,
+                                         kWaitLimitNs)))
+            break;
+          tc_fence_after();
+          issue_pv(x, j);
+          if (!more) mma_commit(o_done(x));
+          if (x == nx - 1) mma_commit(v_empty(s));
+          if (more) {
+            if (x == 0 && !(ok = mbar_wait(k_full(s1), ((j + 1) / C::kStages) & 1, abort_flag,
+                                           kWaitLimitNs)))
+              break;
+            tc_fence_after();
+            issue_s(x, j + 1);
+            if (x == nx - 1) mma_commit(k_empty(s1));
+          }
+        }
       }
       if (!ok) fail();
       // Drain: every MMA issued above has completed once `drain` flips.
       mma_commit(drain);
       mbar_wait(drain, 0, nullptr, kWaitLimitNs);
     }
-  } else {
+  } else if (warp < 4 || it.two) {
     // ------------------------------------------------------ softmax warps
-    // Every tcgen05.ld/st below is executed by all 32 lanes of the warp: the
-    // branches around them are warp-uniform.  Barrier phases: S_j completes
-    // only after PV_{j-2} (in-order MMA pipe), so when PV_{j-1} is awaited on
-    // o_done[(j-1)&1] that barrier is at most one phase behind.
-    const int row = threadIdx.x;                          // 0..127 == TMEM lane
-    const uint32_t lane_addr = tmem + ((uint32_t)(warp * 32) << 16);
+    // Warps 4x..4x+3 own query tile x.  Every tcgen05.ld/st below runs on all
+    // 32 lanes of a warp (the branches around them are warp-uniform).  S_x of
+    // tile j is issued after P_x.V of tile j-1, so once S_x has arrived the
+    // tile's O is quiescent and may be rescaled without a further wait.
+    const int x = warp / 4;
+    const int row = threadIdx.x % 128;                         // TMEM lane
+    const uint32_t lane_addr = tmem + ((uint32_t)((warp % 4) * 32) << 16);
+    const uint32_t sb = lane_addr + C::kTmemS + 128 * x;
+    const uint32_t ob = lane_addr + C::kTmemO + D * x;
     const float sl2 = p.scale_log2;
     constexpr unsigned kAll = 0xffffffffu;
     float m = -INFINITY, l = 0.f;
     bool ok = true;
     for (int j = 0; j < n; ++j) {
-      const int b = j & 1;
-      ok = __all_sync(kAll, mbar_wait(s_full(b), (j >> 1) & 1, abort_flag, kWaitLimitNs));
+      ok = __all_sync(kAll, mbar_wait(s_full(x), j & 1, abort_flag, kWaitLimitNs));
       if (!ok) break;
       tc_fence_after();
       int page_pos, t, valid;
       tile_coords(sp, p.P, it.t_begin + j, page_pos, t, valid);
-      const uint32_t sb = lane_addr + (b ? C::kTmemS1 : C::kTmemS0);
-      uint32_t sr[4][32];
+      float s[128];
+      {
+        uint32_t r0[32], r1[32], r2[32], r3[32];
+        tmem_ld32(sb, r0);
+        tmem_ld32(sb + 32, r1);
+        tmem_ld32(sb + 64, r2);
+        tmem_ld32(sb + 96, r3);
+        tmem_wait_ld();
 #pragma unroll
-      for (int c = 0; c < 4; ++c) tmem_ld32(sb + c * 32, sr[c]);
-      tmem_wait_ld();
-      float mx = -INFINITY;
+        for (int i = 0; i < 32; ++i) {
+          s[i] = __uint_as_float(r0[i]);
+          s[32 + i] = __uint_as_float(r1[i]);
+          s[64 + i] = __uint_as_float(r2[i]);
+          s[96 + i] = __uint_as_float(r3[i]);
+        }
+      }
+      if (valid < kTileN) {
 #pragma unroll
-      for (int c = 0; c < 4; ++c)
+        for (int i = 0; i < 128; ++i) s[i] = i < valid ? s[i] : -INFINITY;
+      }
+      float mx;
+      {
+        float mm[8];
 #pragma unroll
-        for (int i = 0; i < 32; ++i)
-          if (c * 32 + i < valid) mx = fmaxf(mx, __uint_as_float(sr[c][i]));
+        for (int k = 0; k < 8; ++k) mm[k] = fmaxf(s[2 * k], s[2 * k + 1]);
+#pragma unroll
+        for (int i = 8; i < 64; ++i) mm[i % 8] = fmax3(mm[i % 8], s[2 * i], s[2 * i + 1]);
+        mx = fmax3(fmax3(mm[0], mm[1], mm[2]), fmax3(mm[3], mm[4], mm[5]), fmaxf(mm[6], mm[7]));
+      }
       mx *= sl2;
+      // New running max.  The O rescale it may need is done after P is
+      // written (S registers are dead by then) and before P_x is released.
+      bool rescale = false;
+      float alpha = 1.f;
       if (j == 0) {
         m = mx;
       } else if (__any_sync(kAll, mx > m + kRescaleThreshold)) {
-        // O holds the sum over earlier tiles scaled by 2^-m: move it to the new max.
-        ok = __all_sync(kAll, mbar_wait(o_done((j - 1) & 1), ((j - 1) >> 1) & 1, abort_flag,
-                                        kWaitLimitNs));
-        if (!ok) break;
-        tc_fence_after();
         const float mnew = fmaxf(m, mx);
-        const float alpha = ex2(m - mnew);
+        alpha = ex2(m - mnew);
         l *= alpha;
-#pragma unroll
-        for (int c = 0; c < D / 32; ++c) {
-          uint32_t o[32];
-          tmem_ld32(lane_addr + C::kTmemO + c * 32, o);
-          tmem_wait_ld();
-#pragma unroll
-          for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
-          tmem_st32(lane_addr + C::kTmemO + c * 32, o);
-        }
         m = mnew;
+        rescale = true;
       }
-      const float neg_m = -m;
+      const float nm = -m;
+      float la[4] = {0.f, 0.f, 0.f, 0.f}, lb[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
       for (int c = 0; c < 4; ++c) {
         uint32_t pk[16];
 #pragma unroll
         for (int i = 0; i < 16; ++i) {
-          const int col = c * 32 + 2 * i;
-          const float p0 = col < valid ? ex2(fmaf(__uint_as_float(sr[c][2 * i]), sl2, neg_m)) : 0.f;
-          const float p1 =
-              col + 1 < valid ? ex2(fmaf(__uint_as_float(sr[c][2 * i + 1]), sl2, neg_m)) : 0.f;
-          l += p0 + p1;
-          if constexpr (BF16) {
-            __nv_bfloat162 h2 = __floats2bfloat162_rn(p0, p1);
-            pk[i] = *reinterpret_cast<uint32_t*>(&h2);
-          } else {
-            __half2 h2 = __floats2half2_rn(p0, p1);
-            pk[i] = *reinterpret_cast<uint32_t*>(&h2);
-          }
+          float x0, x1, p0, p1;
+          ffma2(x0, x1, s[32 * c + 2 * i], s[32 * c + 2 * i + 1], sl2, sl2, nm, nm);
+#if SVT_EXP_MODE == 1
+          ex2_h2(p0, p1, x0, x1);
+#else
+          p0 = ex2(x0);
+          p1 = ex2(x1);
+#endif
+          fadd2(la[i % 4], lb[i % 4], la[i % 4], lb[i % 4], p0, p1);
+          pk[i] = pack2<BF16>(p0, p1);
         }
-        tmem_st16(sb + c * 16, pk);
+        tmem_st16(sb + 16 * c, pk);
+      }
+      l += (la[0] + lb[0]) + (la[1] + lb[1]) + (la[2] + lb[2]) + (la[3] + lb[3]);
+      if (rescale) {
+        // O holds the sum over earlier tiles scaled by 2^-m_old: move it to 2^-m.
+#pragma unroll
+        for (int c = 0; c < D / 32; ++c) {
+          uint32_t o[32];
+          tmem_ld32(ob + c * 32, o);
+          tmem_wait_ld();
+#pragma unroll
+          for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
+          tmem_st32(ob + c * 32, o);
+        }
       }
       tmem_wait_st();
       tc_fence_before();
-      mbar_arrive(p_full(b));
+      mbar_arrive(p_full(x));
     }
-    if (ok && n > 0)
-      ok = __all_sync(kAll, mbar_wait(o_done((n - 1) & 1), ((n - 1) >> 1) & 1, abort_flag,
-                                      kWaitLimitNs));
+    if (ok && n > 0) ok = __all_sync(kAll, mbar_wait(o_done(x), 0, abort_flag, kWaitLimitNs));
     if (!ok) fail();
     tc_fence_after();
     if (ok && n > 0) {
-      const int r = it.qtile * kTileM + row;
+      const int r = (2 * it.qpair + x) * kTileM + row;
       const bool store = r < sp.nq;
       const float inv = 1.f / l;
       const int grow = sp.q_off + (store ? r : 0);
@@ -349,21 +415,12 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
         for (int c = 0; c < D / 32; ++c) {
           uint32_t o[32];
-          tmem_ld32(lane_addr + C::kTmemO + c * 32, o);
+          tmem_ld32(ob + c * 32, o);
           tmem_wait_ld();
           uint32_t pk[16];
 #pragma unroll
-          for (int i = 0; i < 16; ++i) {
-            const float a0 = __uint_as_float(o[2 * i]) * inv;
-            const float a1 = __uint_as_float(o[2 * i + 1]) * inv;
-            if constexpr (BF16) {
-              __nv_bfloat162 h2 = __floats2bfloat162_rn(a0, a1);
-              pk[i] = *reinterpret_cast<uint32_t*>(&h2);
-            } else {
-              __half2 h2 = __floats2half2_rn(a0, a1);
-              pk[i] = *reinterpret_cast<uint32_t*>(&h2);
-            }
-          }
+          for (int i = 0; i < 16; ++i)
+            pk[i] = pack2<BF16>(__uint_as_float(o[2 * i]) * inv, __uint_as_float(o[2 * i + 1]) * inv);
           if (store) {
             uint4* dst = reinterpret_cast<uint4*>(orow + c * 32);
 #pragma unroll
@@ -378,7 +435,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
         for (int c = 0; c < D / 32; ++c) {
           uint32_t o[32];
-          tmem_ld32(lane_addr + C::kTmemO + c * 32, o);
+          tmem_ld32(ob + c * 32, o);
           tmem_wait_ld();
           if (store) {
 #pragma unroll
@@ -395,7 +452,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     tc_fence_before();
   }
   __syncthreads();
-  if (warp == 5) {
+  if (warp == 9) {
     tc_fence_after();
     tmem_dealloc(tmem, kTmemCols);
   }
@@ -420,6 +477,8 @@ cudaError_t launch_t(const AttnParams& p, const void* tq, const void* tkv, cudaS
 }
 
 }  // namespace
+
+int attn_items_per_stream(int H, int qtiles, int chunks) { return H * ((qtiles + 1) / 2) * chunks; }
 
 cudaError_t launch_attn_sm100(const AttnParams& p, const void* tmap_q, const void* tmap_kv,
                               int dtype, cudaStream_t s) {

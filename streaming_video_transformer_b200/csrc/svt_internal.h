@@ -96,6 +96,8 @@ struct AttnParams {
 };
 
 // Tensor-core (tcgen05 / TMEM) kernel; tensor maps are CUtensorMap (128 bytes each).
+// One work item covers two 128-row query tiles of one (stream, head, KV chunk).
+int attn_items_per_stream(int H, int qtiles, int chunks);
 cudaError_t launch_attn_sm100(const AttnParams& p, const void* tmap_q, const void* tmap_kv,
                               int dtype, cudaStream_t s);
 

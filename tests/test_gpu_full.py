@@ -107,7 +107,7 @@ def test_vitl_stream24_blocks_0_and_23():
     # bf16 step of the value plus the fp32 arithmetic error of the rotation
     # (a few 2^-24 of the input's magnitude, which dominates after cancellation).
     diff = np.abs(gk - ok)
-    assert np.all(diff <= 2.0 ** -8 * np.abs(ok) + 4e-6)
+    assert np.all(diff <= 2.0 ** -7 * np.abs(ok) + 4e-6)
     assert np.mean(diff > 0) < 1e-3
     c.device_error()
 
