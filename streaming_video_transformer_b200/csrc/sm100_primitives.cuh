@@ -254,3 +254,16 @@ __device__ __forceinline__ void ex2_h2(float& y0, float& y1, float x0, float x1)
 }
 }  // namespace sm100
 }  // namespace svt
+
+namespace svt {
+namespace sm100 {
+// Named CTA barriers (ids 1..15; id 0 is __syncthreads).  `count` threads,
+// a multiple of 32, take part: bar_arrive signals without waiting.
+__device__ __forceinline__ void named_bar_sync(uint32_t id, uint32_t count) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
+}
+__device__ __forceinline__ void named_bar_arrive(uint32_t id, uint32_t count) {
+  asm volatile("bar.arrive %0, %1;" ::"r"(id), "r"(count) : "memory");
+}
+}  // namespace sm100
+}  // namespace svt

@@ -744,9 +744,9 @@ int svt_plan(svt_cache* c, const int32_t* qo_len, svt_stream_t) {
   int max_tiles = 0;
   for (int i = 0; i < c->n_streams; ++i)
     if (qo_len[i]) max_tiles = std::max(max_tiles, tiles[i]);
-  // Cost model: one work item covers a pair of 128-row query tiles; a KV tile
-  // costs a pair ~2x(4*128*128*D) flops at ~60% of the per-SM tensor rate.
-  const double pair_tile_us = 2.0 * 4.0 * kTileM * kTileN * c->D / 6.6e6;
+  // Cost model: a work item is one 128-row query tile over a KV chunk; a KV
+  // tile costs 4*128*128*D flops at ~60% of the per-SM tensor rate.
+  const double tile_us = 4.0 * kTileM * kTileN * c->D / 6.6e6 * attn_ctas_per_sm(c->D);
   const double item_us = 2.0;
   std::vector<int> best(c->n_streams, 1);
   double best_t = 1e300;
@@ -765,16 +765,15 @@ int svt_plan(svt_cache* c, const int32_t* qo_len, svt_stream_t) {
         split = true;
         merge_bytes += (double)qo_len[i] * c->H * (c->D + 1) * 4.0 * (cc + 1);
       }
-      const int qp = (qt[i] + 1) / 2;
       for (int h = 0; h < c->H; ++h)
         for (int cix = 0; cix < cc; ++cix)
-          for (int q = 0; q < qp; ++q) {
+          for (int q = 0; q < qt[i]; ++q) {
             int t0 = (int)((int64_t)cix * tiles[i] / cc), t1 = (int)((int64_t)(cix + 1) * tiles[i] / cc);
-            const bool two = 2 * q + 1 < qt[i];
-            cost.push_back(item_us + (t1 - t0) * pair_tile_us * (two ? 1.0 : 0.6));
+            cost.push_back(item_us + (t1 - t0) * tile_us);
           }
     }
-    double t = simulate(cost, c->num_sms) + (split ? 4.0 + merge_bytes / 5.0e6 : 0.0);
+    double t = simulate(cost, c->num_sms * attn_ctas_per_sm(c->D)) +
+               (split ? 4.0 + merge_bytes / 5.0e6 : 0.0);
     if (t < best_t * 0.98) {
       best_t = t;
       best = ch;
