@@ -225,6 +225,30 @@ SVT_API int svt_get_cache_stats(const svt_cache* c, int stream, svt_stats* out);
  * svt_last_error). */
 SVT_API int svt_device_error(svt_cache* c, svt_stream_t s);
 
+/* Paged attention for callers that cannot allocate device memory -- code running while an
+ * allocator is locked or forbidden, inside a framework that owns every device buffer, or under
+ * a fixed memory budget.  The paper has no counterpart: it is a variant of svt_run that needs
+ * no svt_cache and takes its split-KV scratch from a fixed 32 MiB device array inside the
+ * library (held by every GPU that loads the library until the process exits).  It calls no
+ * cudaMalloc/cudaFree.
+ * q, out: device [sum qo_len][H][D] (out in the input dtype, 16-byte aligned); lse: NULL or
+ * device [sum qo_len][H] float32; pool_block: device, one block's pool region
+ * [max_pages][2][page_size][H][D]; indices: DEVICE visible page ids (CSR); indptr
+ * [num_streams+1], last_page_len [num_streams], qo_len [num_streams]: HOST arrays describing
+ * the same table and the query rows per stream.  dtype: SVT_BF16 or SVT_FP16; D: 64 or 128.
+ * num_splits: KV chunks per query tile (0 = chosen automatically within the scratch).  No 2-D
+ * RoPE is applied: pass already rotated queries.
+ * The first call on a device looks up the scratch array's device address (with that device
+ * current); make it before any stream capture.  All calls share the scratch and calls that
+ * overlap on the GPU race on it.
+ * Errors: SVT_EINVAL (bad argument; num_splits whose partials exceed the 32 MiB scratch),
+ * SVT_ECUDA. */
+SVT_API int svt_attention_noalloc(const void* q, void* out, float* lse, const void* pool_block,
+                                  const int32_t* indices, const int32_t* indptr,
+                                  const int32_t* last_page_len, const int32_t* qo_len,
+                                  int num_streams, int max_pages, int page_size, int H, int D,
+                                  int dtype, int num_splits, svt_stream_t s);
+
 /* Message of the last failed call on this thread ("" if none). */
 SVT_API const char* svt_last_error(void);
 

@@ -187,3 +187,25 @@ class PagedKVCache:
 
     def device_error(self, cuda_stream=None) -> None:
         _check(self._lib.svt_device_error(self._h, _stream_handle(cuda_stream)))
+
+
+def attention_noalloc(q, out, pool_block, indices, indptr, last_page_len, qo_len, max_pages,
+                      page_size, lse=None, num_splits=0, cuda_stream=None) -> None:
+    """``svt_attention_noalloc``: paged attention without any device allocation.
+
+    q, out, lse, pool_block (one block's pool region) and indices are device
+    tensors; indptr, last_page_len and qo_len are host sequences.
+    """
+    lib = L.load()
+    H, D = q.shape[1], q.shape[2]
+    dtype = {"torch.bfloat16": L.SVT_BF16, "torch.float16": L.SVT_FP16}[str(q.dtype)]
+    p32 = ctypes.POINTER(ctypes.c_int32)
+    ip = np.ascontiguousarray(indptr, dtype=np.int32)
+    lp = np.ascontiguousarray(last_page_len, dtype=np.int32)
+    ql = np.ascontiguousarray(qo_len, dtype=np.int32)
+    if indices.dtype != _torch().int32:
+        raise ValueError("indices must be int32")
+    _check(lib.svt_attention_noalloc(
+        _ptr(q), _ptr(out), _ptr(lse), _ptr(pool_block), _ptr(indices), ip.ctypes.data_as(p32),
+        lp.ctypes.data_as(p32), ql.ctypes.data_as(p32), len(ql), max_pages, page_size, H, D,
+        dtype, num_splits, _stream_handle(cuda_stream)))

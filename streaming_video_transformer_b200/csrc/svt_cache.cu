@@ -254,6 +254,14 @@ double simulate(const std::vector<double>& item_cost, int num_sms) {
 
 }  // namespace
 
+namespace svt {
+// Records a message for svt_last_error() from another translation unit.
+int report_error(int code, const char* msg) {
+  g_err = msg;
+  return code;
+}
+}  // namespace svt
+
 // =================================================================== C ABI
 extern "C" {
 

@@ -122,4 +122,7 @@ struct SimtParams {
 int simt_rows_per_block(int D);
 cudaError_t launch_attn_simt(const SimtParams& p, int dtype, cudaStream_t s);
 
+// Sets the thread-local message returned by svt_last_error(); returns `code`.
+int report_error(int code, const char* msg);
+
 }  // namespace svt
