@@ -41,6 +41,22 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
       : "memory");
   return ok != 0;
 }
+// As mbar_try_wait, but the thread may be suspended in hardware for up to
+// `suspend_ns` until the phase completes, instead of returning at once: a
+// waiting warp then takes no issue slots from the warps sharing its SM
+// sub-partition.
+__device__ __forceinline__ bool mbar_try_wait_sleep(uint32_t bar, uint32_t parity,
+                                                    uint32_t suspend_ns) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}\n"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity), "r"(suspend_ns)
+      : "memory");
+  return ok != 0;
+}
 __device__ __forceinline__ uint64_t global_timer_ns() {
   uint64_t t;
   asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
@@ -54,12 +70,10 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity,
                                           const volatile int* abort, uint64_t limit_ns) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = global_timer_ns();
-  for (uint32_t it = 1;; ++it) {
-    if (mbar_try_wait(bar, parity)) return true;
-    if ((it & 255u) == 0) {
-      if (abort && *abort) return false;
-      if (global_timer_ns() - t0 > limit_ns) return false;
-    }
+  for (;;) {
+    if (mbar_try_wait_sleep(bar, parity, 1000000u)) return true;
+    if (abort && *abort) return false;
+    if (global_timer_ns() - t0 > limit_ns) return false;
   }
 }
 
@@ -251,19 +265,6 @@ __device__ __forceinline__ void ex2_h2(float& y0, float& y1, float x0, float x1)
       "cvt.f32.f16 %0, lo;\n\tcvt.f32.f16 %1, hi;\n\t}"
       : "=f"(y0), "=f"(y1)
       : "f"(x0), "f"(x1));
-}
-}  // namespace sm100
-}  // namespace svt
-
-namespace svt {
-namespace sm100 {
-// Named CTA barriers (ids 1..15; id 0 is __syncthreads).  `count` threads,
-// a multiple of 32, take part: bar_arrive signals without waiting.
-__device__ __forceinline__ void named_bar_sync(uint32_t id, uint32_t count) {
-  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
-}
-__device__ __forceinline__ void named_bar_arrive(uint32_t id, uint32_t count) {
-  asm volatile("bar.arrive %0, %1;" ::"r"(id), "r"(count) : "memory");
 }
 }  // namespace sm100
 }  // namespace svt

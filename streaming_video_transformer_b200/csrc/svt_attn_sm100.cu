@@ -457,9 +457,13 @@ cudaError_t launch_t(const AttnParams& p, const void* tq, const void* tkv, cudaS
   return cudaGetLastError();
 }
 
+
 }  // namespace
 
-int attn_items_per_stream(int H, int qtiles, int chunks) { return H * qtiles * chunks; }
+int attn_items_per_stream(int H, int D, int qtiles, int chunks) {
+  (void)D;
+  return H * qtiles * chunks;
+}
 
 int attn_ctas_per_sm(int D) { return D == 64 ? 2 : 1; }   // TMEM 256 and < 113 KB smem at D = 64
 

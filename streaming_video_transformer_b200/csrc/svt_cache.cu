@@ -773,11 +773,14 @@ int svt_plan(svt_cache* c, const int32_t* qo_len, svt_stream_t) {
         split = true;
         merge_bytes += (double)qo_len[i] * c->H * (c->D + 1) * 4.0 * (cc + 1);
       }
+      const int per_item = 1;   // one 128-row query tile per work item
+      const int groups = (qt[i] + per_item - 1) / per_item;
       for (int h = 0; h < c->H; ++h)
         for (int cix = 0; cix < cc; ++cix)
-          for (int q = 0; q < qt[i]; ++q) {
+          for (int g = 0; g < groups; ++g) {
             int t0 = (int)((int64_t)cix * tiles[i] / cc), t1 = (int)((int64_t)(cix + 1) * tiles[i] / cc);
-            cost.push_back(item_us + (t1 - t0) * tile_us);
+            const int q_in_item = std::min(per_item, qt[i] - g * per_item);
+            cost.push_back(item_us + (t1 - t0) * tile_us * q_in_item);
           }
     }
     double t = simulate(cost, c->num_sms * attn_ctas_per_sm(c->D)) +
@@ -793,7 +796,7 @@ int svt_plan(svt_cache* c, const int32_t* qo_len, svt_stream_t) {
     StreamPlan& sp = a.s[i];
     sp.chunks = qo_len[i] ? best[i] : 0;
     sp.item_off = items;
-    items += attn_items_per_stream(c->H, sp.qtiles, sp.chunks);
+    items += attn_items_per_stream(c->H, c->D, sp.qtiles, sp.chunks);
     any_split |= sp.chunks > 1;
     info.splits[i] = sp.chunks;
   }

@@ -97,7 +97,7 @@ struct AttnParams {
 
 // Tensor-core (tcgen05 / TMEM) kernel; tensor maps are CUtensorMap (128 bytes each).
 // One work item covers one 128-row query tile of one (stream, head, KV chunk).
-int attn_items_per_stream(int H, int qtiles, int chunks);
+int attn_items_per_stream(int H, int D, int qtiles, int chunks);
 int attn_ctas_per_sm(int D);   // resident CTAs of the tensor-core kernel per SM
 cudaError_t launch_attn_sm100(const AttnParams& p, const void* tmap_q, const void* tmap_kv,
                               int dtype, cudaStream_t s);

@@ -165,7 +165,7 @@ extern "C" SVT_API int svt_attention_noalloc(
     StreamPlan& sp = a.s[i];
     sp.chunks = sp.nq ? std::max(1, std::min(splits, sp.tiles)) : 0;
     sp.item_off = items;
-    items += attn_items_per_stream(H, sp.qtiles, sp.chunks);
+    items += attn_items_per_stream(H, D, sp.qtiles, sp.chunks);
   }
   a.n_streams = num_streams;
   a.total_items = items;
