@@ -37,6 +37,14 @@ WORKLOAD = "vitl_stream24"
 PREFILL = {"vitl_stream24": 72, "vitl_step": 200}
 
 
+# DRAM traffic of one attention launch from the ncu capture summarised in
+# profiles/attn_sm100_vitl_step.md (single ViT-L step, 99,792 visible keys):
+# read 462.6 MB + write 23.6 MB.  Traffic grows with the visible keys, so the
+# bench scales it to the mean key count of its timed frames.  Set to None when
+# the attention kernel changes until a new capture is taken.
+ATTN_TRAFFIC_BYTES, ATTN_TRAFFIC_KEYS = 486.26e6, 99792
+
+
 def _peaks():
     try:
         with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
@@ -421,12 +429,9 @@ def main():
     run_flops = sum(r["flops_per_block"]) / len(r["flops_per_block"])
     achieved = run_flops / (run_avg_ms / 1e3) / 1e12
     traffic = None
-    try:
-        with open(os.path.join(ROOT, "profiles", "attn_traffic.json")) as f:
-            tr = json.load(f)
-            traffic = tr.get("dram_bytes_per_launch")
-    except Exception:
-        pass
+    if ATTN_TRAFFIC_BYTES:
+        keys = [_visible(t + 1, w) for t in range(r["first_timed"], r["last_timed"])]
+        traffic = ATTN_TRAFFIC_BYTES * (sum(keys) / len(keys)) / ATTN_TRAFFIC_KEYS
     cpu = None
     if not args.no_cpu_baseline and world == 1:
         try:
