@@ -193,7 +193,10 @@ SVT_API int svt_read_device_page_table(svt_cache* c, int32_t* indptr, int32_t* i
 
 /* Plans the attention launch once per frame step ([P4] Sec. Plan-Run Execution Workflow):
  * qo_len_per_stream[num_streams] host array of query rows per stream (0 = stream skipped);
- * the query rows of all streams are concatenated in stream order.  Splits each stream's KV
+ * the query rows of all streams are concatenated in stream order.  A stream's query may hold
+ * several frames (the first pass over a clip, [P1] Sec. Step-by-Step Streaming Inference,
+ * step 1): append those frames first, then plan with their rows concatenated; with RoPE the
+ * rows must be whole frames.  Splits each stream's KV
  * range into chunks so that the work items fill the GPU.  Host only; the plan is reused by
  * every block's svt_run until the cache changes.
  * Errors: SVT_ESTATE (table not rebuilt since the last change; a stream with queries but no
@@ -224,6 +227,14 @@ SVT_API int svt_get_cache_stats(const svt_cache* c, int stream, svt_stats* out);
  * of range, a wait that hit its limit).  Returns SVT_OK or SVT_EDEVICE (message in
  * svt_last_error). */
 SVT_API int svt_device_error(svt_cache* c, svt_stream_t s);
+
+/* Failure-detection self-test: runs a one-warp kernel that waits, with the bounded mbarrier
+ * wait every kernel of this library uses, on a barrier that nothing arrives on.  The wait must
+ * give up after limit_us microseconds (1..10^7) and report it; the context stays usable.
+ * Synchronises `s`.  Returns SVT_EDEVICE when the wait gave up as designed (the expected
+ * result), SVT_EINVAL for a bad limit, SVT_ECUDA otherwise.  The pages describe no
+ * failure handling beyond rollback; this covers the kernels' own waits. */
+SVT_API int svt_selftest_wait_limit(int limit_us, svt_stream_t s);
 
 /* Paged attention for callers that cannot allocate device memory -- code running while an
  * allocator is locked or forbidden, inside a framework that owns every device buffer, or under

@@ -132,19 +132,21 @@ class FrameStream:
     def visible_ids(self):
         return visible_frame_ids(len(self.frames), self.S, self.W, self.provisional)
 
-    def visible_kv(self):
+    def visible_kv(self, heads=None):
         """(K, V) of all visible tokens, ``[N, H, D]`` float64, in the order
-        scale patches -> window patches -> specials."""
+        scale patches -> window patches -> specials.  ``heads`` (a slice or
+        index list) restricts the gather to some heads."""
         scale, window, special = self.visible_ids()
+        sel = slice(None) if heads is None else heads
         ks, vs = [], []
         for i in scale + window:
             f = self.frames[i]
             assert f.k_patch is not None, "visible frame lost its patches"
-            ks.append(f.k_patch)
-            vs.append(f.v_patch)
+            ks.append(f.k_patch[:, sel])
+            vs.append(f.v_patch[:, sel])
         for i in special:
-            ks.append(self.frames[i].k_special)
-            vs.append(self.frames[i].v_special)
+            ks.append(self.frames[i].k_special[:, sel])
+            vs.append(self.frames[i].v_special[:, sel])
         return np.concatenate(ks, 0), np.concatenate(vs, 0)
 
     def num_visible_tokens(self) -> int:

@@ -16,7 +16,8 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 CSRC = os.path.join(HERE, "csrc")
 ROOT = os.path.dirname(HERE)
 LIB = os.path.join(HERE, "libsvt.so")
-SOURCES = ["svt_cache.cu", "svt_kernels.cu", "svt_attn_sm100.cu", "svt_noalloc.cu"]
+SOURCES = ["svt_cache.cu", "svt_kernels.cu", "svt_attn_sm100.cu", "svt_noalloc.cu",
+           "svt_selftest.cu"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 
 

@@ -209,3 +209,9 @@ def attention_noalloc(q, out, pool_block, indices, indptr, last_page_len, qo_len
         _ptr(q), _ptr(out), _ptr(lse), _ptr(pool_block), _ptr(indices), ip.ctypes.data_as(p32),
         lp.ctypes.data_as(p32), ql.ctypes.data_as(p32), len(ql), max_pages, page_size, H, D,
         dtype, num_splits, _stream_handle(cuda_stream)))
+
+
+def selftest_wait_limit(limit_us: int, cuda_stream=None) -> None:
+    """``svt_selftest_wait_limit``: raises SvtError(SVT_EDEVICE) when the bounded
+    wait gave up at its limit, which is the expected outcome."""
+    _check(L.load().svt_selftest_wait_limit(int(limit_us), _stream_handle(cuda_stream)))

@@ -729,8 +729,8 @@ int svt_plan(svt_cache* c, const int32_t* qo_len, svt_stream_t) {
     if (qo_len[i] < 0) return fail(SVT_EINVAL, "negative qo_len");
     if (qo_len[i] > 0 && np == 0)
       return fail(SVT_ESTATE, "stream %d has queries but no visible tokens", i);
-    if (c->rope_grid && qo_len[i] && qo_len[i] != c->ns + P)
-      return fail(SVT_EINVAL, "with RoPE each stream's query is one frame (%d rows)", c->ns + P);
+    if (c->rope_grid && qo_len[i] % (c->ns + P))
+      return fail(SVT_EINVAL, "with RoPE each stream's query is whole frames of %d rows", c->ns + P);
     StreamPlan& sp = a.s[i];
     sp.q_off = rows;
     sp.nq = qo_len[i];

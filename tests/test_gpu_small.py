@@ -190,3 +190,83 @@ def test_multi_stream_with_idle_stream():
     for s, rows in ((0, slice(0, w.Nq)), (2, slice(w.Nq, 2 * w.Nq))):
         ref, _ = oracle_out(sts[s], banks[s].oracle(ages[s] - 1)[0])
         assert_close(out[rows], ref, what=f"stream {s}")
+
+
+def test_skip_append_non_keyframe():
+    """A frame that attends without being stored (the upstream skip-append
+    path for non-keyframes): deferred append, attention, rollback.  Its
+    queries see the cache plus its own tokens; afterwards the cache is as
+    before, bit for bit."""
+    w = small_workload(P=48, ns=6, S=2, W=3, H=2, D=64, R=16, blocks=2)
+    c = make_cache(w, max_pages_for(w, [12]))
+    bank = FrameBank(w, 0, 0)
+    st = oracle_stream(w)
+    for t in range(7):
+        q = _step(c, w, bank, t)
+        st.append_frame(*bank.oracle(t)[1:])
+    table, stats = c.get_page_table(), c.get_cache_stats()
+    gk0, gv0 = gather_visible(c, 0, 0)
+    # skip-append frame 7
+    q = _step(c, w, bank, 7, deferred=True)
+    st.append_frame(*bank.oracle(7)[1:], deferred=True)
+    ref, _ = oracle_out(st, bank.oracle(7)[0])
+    assert_close(c.run(0, q), ref, what="skip-append frame")
+    c.rollback_last_frame()
+    c.set_defer_eviction(False)
+    st.rollback_last_frame()
+    for a, b in zip(table, c.get_page_table()):
+        assert np.array_equal(a, b)
+    assert c.get_cache_stats() == stats
+    c.build_visible_page_table()
+    gk1, gv1 = gather_visible(c, 0, 0)
+    assert np.array_equal(gk0, gk1) and np.array_equal(gv0, gv1)
+    # the next stored frame sees exactly the cache it would have seen
+    q = _step(c, w, bank, 8)
+    st.append_frame(*bank.oracle(8)[1:])
+    ref, _ = oracle_out(st, bank.oracle(8)[0])
+    assert_close(c.run(0, q), ref, what="frame after skip-append")
+
+
+def test_multi_frame_first_pass_with_rope():
+    """First pass over a clip: several frames appended, then all of their
+    queries attend at once (no causal mask among them)."""
+    w = small_workload(P=16, ns=6, S=4, W=4, H=2, D=64, R=8, rope_grid=4)
+    F = 3
+    c = make_cache(w, max_pages_for(w, [F]), max_qo_len=F * w.Nq)
+    bank = FrameBank(w, 0, 0)
+    st = oracle_stream(w)
+    for t in range(F):
+        c.append_frame(0, *bank.device(t)[1:])
+        c.evict_frames()
+        st.append_frame(*bank.oracle(t)[1:])
+    c.build_visible_page_table()
+    c.plan([F * w.Nq])
+    q = torch.cat([bank.device(t)[0] for t in range(F)])
+    q64 = np.concatenate([bank.oracle(t)[0] for t in range(F)])
+    ref, _ = oracle_out(st, q64)
+    assert_close(c.run(0, q), ref, what="first pass")
+    assert_close(c.run(0, q, force_fp32=True), ref, fp32=True, what="first pass fp32")
+
+
+def test_bounded_wait_gives_up_and_context_stays_usable():
+    """Failure detection without a fault: a kernel waits on an mbarrier that
+    nothing arrives on; the bounded wait gives up and reports, and the GPU
+    keeps working."""
+    import time
+    from streaming_video_transformer_b200 import _lib
+    from streaming_video_transformer_b200.cache import SvtError, selftest_wait_limit
+    t0 = time.perf_counter()
+    with pytest.raises(SvtError) as e:
+        selftest_wait_limit(20000)                 # 20 ms
+    assert e.value.code == _lib.SVT_EDEVICE
+    assert time.perf_counter() - t0 < 5.0
+    w = WORKLOADS["tiny_stream"]
+    c = make_cache(w, max_pages_for(w, [3]))
+    bank = FrameBank(w, 0, 0)
+    st = oracle_stream(w)
+    for t in range(3):
+        q = _step(c, w, bank, t)
+        st.append_frame(*bank.oracle(t)[1:])
+    ref, _ = oracle_out(st, bank.oracle(2)[0])
+    assert_close(c.run(0, q), ref, what="after the self-test")
+    c.device_error()
