@@ -35,6 +35,8 @@ METRIC = "streamed frames/s (24-block paged attn) and attn TFLOP/s as % of bf16 
 WORKLOAD = "vitl_stream24"
 # frames appended (no attention) before the warm-up steps
 PREFILL = {"vitl_stream24": 72, "vitl_step": 200}
+# further workloads measured by run_secondary (one JSON line each)
+SECONDARY = ("tiny_stream", "ragged4", "rollback10k")
 
 
 # DRAM traffic of one attention launch from the ncu capture summarised in
@@ -287,6 +289,128 @@ def run_gpu(args, rank, world, local_rank):
                 kernels_per_step=kernels_per_step, first_timed=first_timed, last_timed=t_frame)
 
 
+# ----------------------------------------------------- secondary workloads
+def run_secondary(args):
+    """The other workloads of the scheme, each timed with CUDA events:
+    tiny_stream -- the whole 12-frame stream (append, evict, build, plan, run
+                   per frame), repeated; ragged4 -- one batched run over four
+                   streams aged 10/70/300/2000 (fp16, D=128); rollback10k --
+                   10,000 offered frames, every 3rd deferred and rejected with
+                   p=0.3, in bf16, and a sample of late frames with an fp32 pool."""
+    import torch
+    from dataclasses import replace
+
+    from streaming_video_transformer_b200.cache import PagedKVCache
+    from streaming_video_transformer_b200.inputs import WORKLOADS, frame_qkv, keyframe_decisions
+
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    w = WORKLOADS[args.workload]
+    ev = lambda: torch.cuda.Event(enable_timing=True)
+    line = {"impl": "svt", "workload": args.workload, "n_gpus": 1, "data": "synthetic",
+            "dtype": w.dtype, "config": _config(w)}
+    flops_of = lambda nq, nk, H, D: 4.0 * nq * nk * H * D
+
+    def make(wl, frames, streams=1):
+        mp = streams * (wl.S + wl.W + 1) + sum(math.ceil(f * wl.ns / wl.P) for f in frames) + 2 * streams
+        return PagedKVCache(mp, wl.P, wl.H, wl.D, wl.W, wl.S, num_special=wl.ns, num_streams=streams,
+                            dtype=wl.dtype, max_qo_len=streams * wl.Nq, device=dev)
+
+    if args.workload == "tiny_stream":
+        c = make(w, [w.frames])
+        fr = [[x.to(dev) for x in frame_qkv(w, 0, 0, t)] for t in range(w.frames)]
+        out = torch.empty_like(fr[0][0])
+
+        def stream_once():
+            c.reset()
+            for t in range(w.frames):
+                q, k, v = fr[t]
+                c.append_frame(0, k, v)
+                c.evict_frames()
+                c.build_visible_page_table()
+                c.plan([w.Nq])
+                c.run(0, q, out=out)
+        for _ in range(args.warmup):
+            stream_once()
+        torch.cuda.synchronize()
+        a, b = ev(), ev()
+        a.record()
+        for _ in range(args.steps):
+            stream_once()
+        b.record()
+        torch.cuda.synchronize()
+        ms = a.elapsed_time(b)
+        line.update(metric="frames/s (12-frame stream, full frame step)",
+                    value=args.steps * w.frames / (ms / 1e3), unit="frames/s",
+                    us_per_frame=1e3 * ms / (args.steps * w.frames), steps=args.steps)
+    elif args.workload == "ragged4":
+        ages = list(w.ages)
+        c = make(w, ages, streams=4)
+        for s_, age in enumerate(ages):
+            fr = [[x.to(dev) for x in frame_qkv(w, 0, s_, i)] for i in range(min(w.R, age))]
+            for t in range(age):
+                c.append_frame(0, fr[t % len(fr)][1], fr[t % len(fr)][2], stream=s_)
+                c.evict_frames(s_)
+        c.build_visible_page_table()
+        c.plan([w.Nq] * 4)
+        info = c.plan_info()
+        q = torch.cat([frame_qkv(w, 0, s_, 0)[0] for s_ in range(4)]).to(dev)
+        out = torch.empty_like(q)
+        for _ in range(args.warmup):
+            c.run(0, q, out=out)
+        torch.cuda.synchronize()
+        times = []
+        for _ in range(args.steps):
+            a, b = ev(), ev()
+            a.record()
+            c.run(0, q, out=out)
+            b.record()
+            times.append((a, b))
+        torch.cuda.synchronize()
+        ms = statistics.median(x.elapsed_time(y) for x, y in times)
+        flops = sum(flops_of(w.Nq, nk, w.H, w.D) for nk in info["kv_tokens"])
+        line.update(metric="batched run over 4 ragged streams", value=flops / (ms / 1e3) / 1e12,
+                    unit="TFLOP/s", ms_per_run=ms, kv_tokens=info["kv_tokens"],
+                    splits=info["splits"], steps=args.steps)
+    else:   # rollback10k
+        dec = keyframe_decisions(w, w.frames)
+        n_acc = sum(1 for d, r in dec if not r)
+        res = {}
+        for mode in ("bf16", "fp32"):
+            wm = w if mode == "bf16" else replace(w, dtype="fp32")
+            c = make(wm, [n_acc + 1])
+            fr = [[x.to(dev) for x in frame_qkv(wm, 0, 0, i)] for i in range(4)]
+            out = torch.empty((w.Nq, w.H, w.D), dtype=torch.float32 if mode == "fp32" else torch.bfloat16,
+                              device=dev)
+            timed = range(w.frames) if mode == "bf16" else range(w.frames - 20, w.frames)
+            flops = 0.0
+            a, b = ev(), ev()
+            for t, (deferred, rejected) in enumerate(dec):
+                q, k, v = fr[t % 4]
+                c.set_defer_eviction(deferred)
+                c.append_frame(0, k, v)
+                c.evict_frames()
+                if t == timed[0]:
+                    torch.cuda.synchronize()
+                    a.record()
+                if t in timed:
+                    c.build_visible_page_table()
+                    c.plan([w.Nq])
+                    c.run(0, q, out=out, force_fp32=(mode == "fp32"))
+                    flops += flops_of(w.Nq, c.plan_info()["kv_tokens"][0], w.H, w.D)
+                if deferred:
+                    (c.rollback_last_frame if rejected else c.execute_deferred_eviction)()
+            b.record()
+            torch.cuda.synchronize()
+            ms = a.elapsed_time(b)
+            res[mode] = {"frames": len(timed), "frames_per_s": len(timed) / (ms / 1e3),
+                         "tflops": flops / (ms / 1e3) / 1e12}
+        line.update(metric="frames/s over the 10,000-frame stream with rollbacks",
+                    value=res["bf16"]["frames_per_s"], unit="frames/s", modes=res,
+                    accepted_frames=n_acc)
+    print(json.dumps(line), flush=True)
+
+
 # ------------------------------------------------------------- CPU oracle
 def oracle_block_frame_seconds(w, t_frames, rows=None, heads=None):
     """Times the oracle on one block at a cache holding t_frames frames."""
@@ -399,8 +523,9 @@ def main():
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", default="svt", choices=["svt", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--workload", default=WORKLOAD, choices=sorted(PREFILL),
-                    help="vitl_step (1 block, no RoPE) is the small case used for profiling")
+    ap.add_argument("--workload", default=WORKLOAD, choices=sorted(PREFILL) + list(SECONDARY),
+                    help="vitl_step (1 block, no RoPE) is the small case used for profiling; "
+                         "tiny_stream, ragged4 and rollback10k print their own metric")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
@@ -411,6 +536,11 @@ def main():
     if args.impl == "reference":
         if rank == 0:
             print(json.dumps(run_reference(args)), flush=True)
+        return
+    if args.workload in SECONDARY:
+        from streaming_video_transformer_b200.build import build
+        build()
+        run_secondary(args)
         return
 
     if world > 1:
