@@ -608,8 +608,8 @@ def main():
         "cpu_baseline": cpu,
         "e2e": {"value": e2e_fps, "unit": "frames/s", "h2d_bytes_per_step": r["h2d_per_step"],
                 "d2h_bytes_per_step": r["d2h_per_step"], "steps": r["e2e_steps"],
-                "note": "inputs of all 24 blocks copied from pinned host memory each frame on a "
-                        "copy stream (double-buffered), last block's output read back"},
+                "note": f"inputs of all {w.blocks} blocks copied from pinned host memory each frame on "
+                        "a copy stream (double-buffered), last block's output read back"},
         "gpu_launches": r["kernels_per_step"] * args.steps,
         "clocks": r["clocks"],
     }
