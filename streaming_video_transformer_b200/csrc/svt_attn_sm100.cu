@@ -292,12 +292,21 @@ __global__ void __launch_bounds__(kThreads, 2)
     constexpr unsigned kAll = 0xffffffffu;
     float m = -INFINITY, l = 0.f;
     bool ok = true;
+    // Position of the current tile in the visible table, advanced by one
+    // tile per iteration (no divisions on the per-tile path).
+    const int tpp = (p.P + kTileN - 1) / kTileN;
+    const int last_page = sp.n_pages - 1, lpl = sp.lpl, P = p.P;
+    int page_pos, t, valid;
+    tile_coords(sp, P, it.t_begin, page_pos, t, valid);
     for (int j = 0; j < n && ok; ++j) {
+      valid = min(kTileN, (page_pos < last_page ? P : lpl) - t * kTileN);
+      if (++t == tpp && page_pos < last_page) {
+        t = 0;
+        ++page_pos;
+      }
       ok = __all_sync(kAll, mbar_wait(s_full, j & 1, abort_flag, kWaitLimitNs));
       if (!ok) break;
       tc_fence_after();
-      int page_pos, t, valid;
-      tile_coords(sp, p.P, it.t_begin + j, page_pos, t, valid);
       float s[128];
       {
         uint32_t r0[32], r1[32], r2[32], r3[32];
@@ -358,10 +367,13 @@ __global__ void __launch_bounds__(kThreads, 2)
         // behind: P_{j-1} was only written after P_{j-2}.V_{j-2} completed.
         if (c == 0 && j > 0) {
           ok = __all_sync(kAll, mbar_wait(o_done, (j - 1) & 1, abort_flag, kWaitLimitNs));
-          if (ok) tc_fence_after();
+          tc_fence_after();
         }
         // P (16-bit pairs) of score columns 32c..32c+31 -> P columns 16c..16c+15.
-        if (ok) tmem_st16(pb + 16 * c, pk);
+        // Unconditional, so that the exponentials of the next chunk can be
+        // scheduled across it; after a failed wait it only writes this CTA's
+        // own TMEM columns before the loop is left.
+        tmem_st16(pb + 16 * c, pk);
       }
       if (!ok) break;
       l += (la[0] + la[1]) + (la[2] + la[3]);
