@@ -56,6 +56,20 @@ def _peaks():
         return 1590.0, 1400.0, 6650.0, "fallback"
 
 
+L2_BYTES = 126 * 2**20
+
+
+def _l2_note(w):
+    """Visible K/V bytes per block at the last frame, against the L2 size."""
+    ages = w.ages or (w.frames,)
+    elem = 4 if w.dtype == "fp32" else 2
+    tokens = sum(min(a, w.S + w.W) * w.P + w.ns * a for a in ages)
+    kv = tokens * w.H * w.D * 2 * elem
+    if kv > L2_BYTES:
+        return f"inputs larger than L2 ({kv / 1e6:.0f} MB of visible K/V per block)"
+    return f"visible K/V ({kv / 1e3:.0f} KB per block) fits in L2: timings are L2-resident"
+
+
 def _config(w, extra=None):
     desc = (f"{w.name}: {w.blocks} block(s), H={w.H}, D={w.D}, P=page={w.P}, {w.ns} special/frame, "
             f"S={w.S}, W={w.W}, " + (f"2-D RoPE {w.rope_grid}x{w.rope_grid} theta={w.rope_theta:g}, "
@@ -63,7 +77,7 @@ def _config(w, extra=None):
     cfg = {"workload": desc,
            "blocks": w.blocks, "heads": w.H, "head_dim": w.D, "page_size": w.P,
            "num_special": w.ns, "scale_frames": w.S, "sliding_window": w.W,
-           "parallelism": "replicas", "l2": "inputs larger than L2 (437 MB pool per block)"}
+           "parallelism": "replicas", "l2": _l2_note(w)}
     if extra:
         cfg.update(extra)
     return cfg
