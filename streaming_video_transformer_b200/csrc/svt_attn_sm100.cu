@@ -45,7 +45,9 @@ using namespace sm100;
 
 constexpr int kThreads = 192;
 constexpr uint64_t kWaitLimitNs = 2000000000ull;   // 2 s
-constexpr float kRescaleThreshold = 8.0f;          // log2 units
+// A tile's P row is accepted while its sum stays at or below this bound, so
+// that every P value is at most 2^8 (within fp16's range for the P.V MMA).
+constexpr float kRowSumBound = 256.0f;
 
 template <int D>
 struct Cfg {
@@ -122,7 +124,7 @@ __device__ __forceinline__ uint32_t pack2(float lo, float hi) {
 }
 
 template <int D, bool BF16>
-__global__ void __launch_bounds__(kThreads, 2)
+__global__ void __launch_bounds__(kThreads, D == 64 ? 2 : 1)
     attn_sm100_kernel(const __grid_constant__ CUtensorMap tmap_q,
                       const __grid_constant__ CUtensorMap tmap_kv,
                       const __grid_constant__ AttnParams p) {
@@ -290,7 +292,11 @@ __global__ void __launch_bounds__(kThreads, 2)
     const uint32_t ob = lane_addr + C::kTmemO;
     const float sl2 = p.scale_log2;
     constexpr unsigned kAll = 0xffffffffu;
-    float m = -INFINITY, l = 0.f;
+    // Running maximum m (log2 units): very negative but finite at the start,
+    // so that the first tile's exponentials overflow to +inf, its row-sum
+    // test fails and it is computed against its exact maximum; masked (-inf)
+    // scores still give 0.
+    float m = -1e30f, l = 0.f;
     bool ok = true;
     // Position of the current tile in the visible table, advanced by one
     // tile per iteration (no divisions on the per-tile path).
@@ -329,53 +335,79 @@ __global__ void __launch_bounds__(kThreads, 2)
 #pragma unroll
         for (int i = 0; i < 128; ++i) s[i] = i < valid ? s[i] : -INFINITY;
       }
-      float mx;
-      {
-        float mm[8];
-#pragma unroll
-        for (int k = 0; k < 8; ++k) mm[k] = fmaxf(s[2 * k], s[2 * k + 1]);
-#pragma unroll
-        for (int i = 8; i < 64; ++i) mm[i % 8] = fmax3(mm[i % 8], s[2 * i], s[2 * i + 1]);
-        mx = fmax3(fmax3(mm[0], mm[1], mm[2]), fmax3(mm[3], mm[4], mm[5]), fmaxf(mm[6], mm[7]));
-      }
-      mx *= sl2;
-      bool rescale = false;
-      float alpha = 1.f;
-      if (j == 0) {
-        m = mx;
-      } else if (__any_sync(kAll, mx > m + kRescaleThreshold)) {
-        const float mnew = fmaxf(m, mx);
-        alpha = ex2(m - mnew);
-        l *= alpha;
-        m = mnew;
-        rescale = true;
-      }
-      const float nm = -m;
+      // The exponentials are taken against the running maximum m of the
+      // earlier tiles, without a reduction over this tile first.  P values
+      // are non-negative, so the row sum bounds each of them: while it stays
+      // at or below kRowSumBound, P, l and O are consistent with m and the
+      // tile stands as computed (online softmax is exact for any m; the
+      // bound only keeps P in range).  Otherwise (the first tile, or a score
+      // more than one log2 unit above m) the tile's maximum is reduced, m is
+      // raised to it, and the tile is recomputed.
       float la[4] = {0.f, 0.f, 0.f, 0.f};
+      {
+        const float nm = -m;
 #pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        uint32_t pk[16];
+        for (int c = 0; c < 4; ++c) {
+          uint32_t pk[16];
 #pragma unroll
-        for (int i = 0; i < 16; ++i) {
-          const float p0 = ex2(fmaf(s[32 * c + 2 * i], sl2, nm));
-          const float p1 = ex2(fmaf(s[32 * c + 2 * i + 1], sl2, nm));
-          la[i % 4] += p0 + p1;
-          pk[i] = pack2<BF16>(p0, p1);
+          for (int i = 0; i < 16; ++i) {
+            const float p0 = ex2(fmaf(s[32 * c + 2 * i], sl2, nm));
+            const float p1 = ex2(fmaf(s[32 * c + 2 * i + 1], sl2, nm));
+            la[i % 4] += p0 + p1;
+            pk[i] = pack2<BF16>(p0, p1);
+          }
+          // P_{j-1}.V_{j-1} must have read the P columns (and finished
+          // updating O) before P_j is written and O rescaled.  o_done is at
+          // most one phase behind: P_{j-1} was only written after
+          // P_{j-2}.V_{j-2} completed.
+          if (c == 0 && j > 0) {
+            ok = __all_sync(kAll, mbar_wait(o_done, (j - 1) & 1, abort_flag, kWaitLimitNs));
+            tc_fence_after();
+          }
+          // P (16-bit pairs) of score columns 32c..32c+31 -> P columns
+          // 16c..16c+15.  Unconditional, so that the exponentials of the next
+          // chunk can be scheduled across it; after a failed wait it only
+          // writes this CTA's own TMEM columns before the loop is left.
+          tmem_st16(pb + 16 * c, pk);
         }
-        // P_{j-1}.V_{j-1} must have read the P columns (and finished updating
-        // O) before P_j is written and O rescaled.  o_done is at most one phase
-        // behind: P_{j-1} was only written after P_{j-2}.V_{j-2} completed.
-        if (c == 0 && j > 0) {
-          ok = __all_sync(kAll, mbar_wait(o_done, (j - 1) & 1, abort_flag, kWaitLimitNs));
-          tc_fence_after();
-        }
-        // P (16-bit pairs) of score columns 32c..32c+31 -> P columns 16c..16c+15.
-        // Unconditional, so that the exponentials of the next chunk can be
-        // scheduled across it; after a failed wait it only writes this CTA's
-        // own TMEM columns before the loop is left.
-        tmem_st16(pb + 16 * c, pk);
       }
       if (!ok) break;
+      bool rescale = false;
+      float alpha = 1.f;
+      if (__any_sync(kAll, (la[0] + la[1]) + (la[2] + la[3]) > kRowSumBound)) {
+        float mm[4];
+#pragma unroll
+        for (int k = 0; k < 4; ++k) mm[k] = fmaxf(s[2 * k], s[2 * k + 1]);
+#pragma unroll
+        for (int i = 4; i < 64; ++i) mm[i % 4] = fmax3(mm[i % 4], s[2 * i], s[2 * i + 1]);
+        const float mx = fmaxf(fmaxf(mm[0], mm[1]), fmaxf(mm[2], mm[3])) * sl2;
+        if (__any_sync(kAll, mx > m)) {
+          // Recompute this tile against the new maximum and rescale the
+          // state of the earlier tiles (none for the first tile: l is 0 and
+          // O is overwritten by the first P.V).  A row sum above the bound
+          // implies a P above 2, so this branch always raises m.
+          const float mnew = fmaxf(m, mx);
+          alpha = ex2(m - mnew);
+          l *= alpha;
+          m = mnew;
+          rescale = j > 0;
+          const float nm = -m;
+          la[0] = la[1] = la[2] = la[3] = 0.f;
+          tmem_wait_st();
+#pragma unroll
+          for (int c = 0; c < 4; ++c) {
+            uint32_t pk[16];
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+              const float p0 = ex2(fmaf(s[32 * c + 2 * i], sl2, nm));
+              const float p1 = ex2(fmaf(s[32 * c + 2 * i + 1], sl2, nm));
+              la[i % 4] += p0 + p1;
+              pk[i] = pack2<BF16>(p0, p1);
+            }
+            tmem_st16(pb + 16 * c, pk);
+          }
+        }
+      }
       l += (la[0] + la[1]) + (la[2] + la[3]);
       if (rescale) {
         // O holds the sum over earlier tiles scaled by 2^-m_old.
