@@ -270,3 +270,51 @@ def test_bounded_wait_gives_up_and_context_stays_usable():
     ref, _ = oracle_out(st, bank.oracle(2)[0])
     assert_close(c.run(0, q), ref, what="after the self-test")
     c.device_error()
+
+
+@pytest.mark.parametrize("splits", [1, 16])
+@pytest.mark.parametrize("dtype", ["bf16", "fp16"])
+@pytest.mark.parametrize("jump", [3.0, 60.0, 150.0, -150.0])
+def test_row_max_jumps_in_later_tiles(dtype, jump, splits):
+    """Keys whose scores sit `jump` log2 units above (or below) the rest
+    appear in a late patch page and among the last special tokens (the
+    partial last page), so that the running maximum taken from the earlier
+    tiles is exceeded mid-row: by a little, by enough that the speculative
+    exponentials exceed 2^8, and by enough that they overflow to +inf.
+    With one KV chunk per row the jumps land in the 6th and 9th of 9 tiles
+    of one CTA; with the planner's splits they may open a chunk."""
+    w = small_workload(P=256, ns=6, S=1, W=3, H=2, D=64, frames=5, R=5, dtype=dtype)
+    tdt = w.torch_dtype
+    g = torch.Generator().manual_seed(5150)
+    u = torch.zeros(w.D)
+    u[7] = 1.0
+    beta = 4.0                                     # shared q component along u
+    alpha = jump * np.sqrt(w.D) / (np.log2(np.e) * beta)
+    frames = []
+    for t in range(w.frames):
+        k = torch.randn((w.Nq, w.H, w.D), generator=g) / np.sqrt(w.D)
+        v = torch.randn((w.Nq, w.H, w.D), generator=g)
+        if t == w.frames - 2:
+            k[w.ns + 100] = alpha * u              # a patch key of a late window page
+        if t == w.frames - 1:
+            k[2] = alpha * u                       # a special key on the last page
+        frames.append((k.to(tdt), v.to(tdt)))
+    q = (torch.randn((w.Nq, w.H, w.D), generator=g) / np.sqrt(w.D) + beta * u).to(tdt)
+    c = make_cache(w, max_pages_for(w, [w.frames]), max_splits=splits)
+    st = oracle_stream(w)
+    for k, v in frames:
+        c.append_frame(0, k.cuda(), v.cuda())
+        c.evict_frames()
+        st.append_frame(k.double().numpy(), v.double().numpy())
+    c.build_visible_page_table()
+    c.plan([w.Nq])
+    if splits == 1:
+        info = c.plan_info()
+        assert info["splits"] == [1] and info["kv_tiles"] == [9]
+    ref, lse_ref = oracle_out(st, q.double().numpy())
+    lse = torch.empty((w.Nq, w.H), dtype=torch.float32, device="cuda")
+    out = c.run(0, q.cuda(), lse=lse)
+    assert_close(out, ref, what=f"{dtype} jump {jump}")
+    np.testing.assert_allclose(lse.cpu().numpy(), lse_ref, rtol=1e-3, atol=2e-2)
+    assert_close(c.run(0, q.cuda(), force_fp32=True), ref, fp32=True, what=f"fp32 jump {jump}")
+    c.device_error()
