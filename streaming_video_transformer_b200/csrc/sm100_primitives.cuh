@@ -221,50 +221,12 @@ __device__ __forceinline__ float ex2(float x) {
   return y;
 }
 
-}  // namespace sm100
-}  // namespace svt
-
-namespace svt {
-namespace sm100 {
-// ------------------------------------------------- packed fp32 arithmetic
-// d = a * b + c on two fp32 lanes at once (one f32x2 instruction).
-__device__ __forceinline__ void ffma2(float& d0, float& d1, float a0, float a1, float b0, float b1,
-                                      float c0, float c1) {
-  asm("{\n\t.reg .b64 ra, rb, rc, rd;\n\t"
-      "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\tmov.b64 rc, {%6, %7};\n\t"
-      "fma.rn.f32x2 rd, ra, rb, rc;\n\tmov.b64 {%0, %1}, rd;\n\t}"
-      : "=f"(d0), "=f"(d1)
-      : "f"(a0), "f"(a1), "f"(b0), "f"(b1), "f"(c0), "f"(c1));
-}
-__device__ __forceinline__ void fadd2(float& d0, float& d1, float a0, float a1, float b0, float b1) {
-  asm("{\n\t.reg .b64 ra, rb, rd;\n\t"
-      "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
-      "add.rn.f32x2 rd, ra, rb;\n\tmov.b64 {%0, %1}, rd;\n\t}"
-      : "=f"(d0), "=f"(d1)
-      : "f"(a0), "f"(a1), "f"(b0), "f"(b1));
-}
+// 3-input maximum (one instruction on sm_100).
 __device__ __forceinline__ float fmax3(float a, float b, float c) {
   float d;
   asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
   return d;
 }
-}  // namespace sm100
-}  // namespace svt
 
-namespace svt {
-namespace sm100 {
-// 2^x for two fp32 inputs using the packed half-precision MUFU path (two
-// results per instruction): x is rounded to f16, exponentiated in f16 and
-// widened back to fp32.  Relative error is dominated by the f16 rounding of
-// x (<= 2^-11 |x| ln 2), below the 16-bit rounding P receives afterwards.
-__device__ __forceinline__ void ex2_h2(float& y0, float& y1, float x0, float x1) {
-  asm("{\n\t.reg .b32 h;\n\t.reg .b16 lo, hi;\n\t"
-      "cvt.rn.f16x2.f32 h, %3, %2;\n\t"
-      "ex2.approx.f16x2 h, h;\n\t"
-      "mov.b32 {lo, hi}, h;\n\t"
-      "cvt.f32.f16 %0, lo;\n\tcvt.f32.f16 %1, hi;\n\t}"
-      : "=f"(y0), "=f"(y1)
-      : "f"(x0), "f"(x1));
-}
 }  // namespace sm100
 }  // namespace svt

@@ -753,7 +753,9 @@ int svt_plan(svt_cache* c, const int32_t* qo_len, svt_stream_t) {
   for (int i = 0; i < c->n_streams; ++i)
     if (qo_len[i]) max_tiles = std::max(max_tiles, tiles[i]);
   // Cost model: a work item is one 128-row query tile over a KV chunk; a KV
-  // tile costs 4*128*128*D flops at ~60% of the per-SM tensor rate.
+  // tile costs 4*128*128*D flops at 6.6 TFLOP/s per SM (a round figure near
+  // what the kernel sustains; only its ratio to the fixed per-item and merge
+  // costs steers the choice), shared by the CTAs resident on one SM.
   const double tile_us = 4.0 * kTileM * kTileN * c->D / 6.6e6 * attn_ctas_per_sm(c->D);
   const double item_us = 2.0;
   std::vector<int> best(c->n_streams, 1);
