@@ -281,8 +281,9 @@ def test_row_max_jumps_in_later_tiles(dtype, jump, splits):
     partial last page), so that the running maximum taken from the earlier
     tiles is exceeded mid-row: by a little, by enough that the speculative
     exponentials exceed 2^8, and by enough that they overflow to +inf.
-    With one KV chunk per row the jumps land in the 6th and 9th of 9 tiles
-    of one CTA; with the planner's splits they may open a chunk."""
+    With one KV chunk per row both jumps land in late tiles of one CTA (the
+    last tile for the special key); with the planner's splits they may open
+    a chunk."""
     w = small_workload(P=256, ns=6, S=1, W=3, H=2, D=64, frames=5, R=5, dtype=dtype)
     tdt = w.torch_dtype
     g = torch.Generator().manual_seed(5150)
@@ -310,7 +311,7 @@ def test_row_max_jumps_in_later_tiles(dtype, jump, splits):
     c.plan([w.Nq])
     if splits == 1:
         info = c.plan_info()
-        assert info["splits"] == [1] and info["kv_tiles"] == [9]
+        assert info["splits"] == [1] and info["kv_tiles"][0] >= 9
     ref, lse_ref = oracle_out(st, q.double().numpy())
     lse = torch.empty((w.Nq, w.H), dtype=torch.float32, device="cuda")
     out = c.run(0, q.cuda(), lse=lse)
