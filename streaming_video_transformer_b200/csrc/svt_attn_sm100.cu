@@ -23,10 +23,12 @@
 //               S_{j+1} is issued as soon as the softmax has read S_j, so the
 //               tensor cores compute it while the softmax exponentiates S_j.
 //   warps 0-3   softmax: thread r owns query row r (TMEM lane r): reads S_j
-//               and releases it, keeps the running max and sum in the log2
-//               domain, writes P_j as 16-bit pairs once P_{j-1}.V_{j-1} has
-//               completed (which also leaves O quiescent for the lazy rescale
-//               done when the max grew by more than 2^8).
+//               and releases it, exponentiates in the log2 domain against the
+//               running maximum of the earlier tiles (no reduction over the
+//               tile first), writes P_j as 16-bit pairs once P_{j-1}.V_{j-1}
+//               has completed (which also leaves O quiescent for a rescale),
+//               and recomputes the tile against its exact maximum only when
+//               the row sum of P_j exceeds 2^8 (always on the first tile).
 // The exponential unit is the bound at D = 64 (one exp per 256 MMA flops);
 // the two CTAs on an SM keep it busy between each other's phases.
 // Split-KV chunks write fp32 partials and LSE; a merge kernel combines them.
