@@ -213,6 +213,8 @@ SVT_API int svt_get_plan_info(const svt_cache* c, svt_plan_info* out);
  * q, out: [sum qo_len][H][D] device arrays; out is in the cache dtype, or float32 when
  * force_fp32 != 0 or the cache dtype is SVT_FP32.  lse: NULL or [sum qo_len][H] float32
  * natural-log log-sum-exp of the scaled scores.
+ * Tensor-core path (bf16/fp16 cache): scores and O accumulate in fp32 (TMEM); the softmax
+ * numerators are rounded to the cache dtype before P.V and stay at or below 2^8 (fp16-safe).
  * force_fp32 = 1 computes with fp32 FMA instead of the tensor cores (the upstream's
  * force_fp32 validation path, [P2] Sec. Memory Efficiency Analysis).
  * Errors: SVT_ESTATE (no valid plan; block not yet appended for the current frame of a
