@@ -53,25 +53,33 @@ constexpr float kRowSumBound = 256.0f;
 
 template <int D>
 struct Cfg {
+  static constexpr int TN = attn_tile_n(D);                    // KV tokens per tile
   static constexpr int kRegions = D / 64;                      // 64-feature swizzle columns
-  static constexpr uint32_t kTileBytes = kTileN * D * 2;       // one K, V or Q tile
-  static constexpr uint32_t kRegionBytes = kTileN * 128;       // 128 rows x 128 bytes
-  // K and V rings; D = 64 keeps a CTA under half an SM's shared memory.
+  static constexpr uint32_t kQBytes = kTileM * D * 2;          // the Q tile
+  static constexpr uint32_t kQRegionBytes = kTileM * 128;      // 128 rows x 128 bytes
+  static constexpr uint32_t kKVBytes = TN * D * 2;             // one K or V tile
+  static constexpr uint32_t kKVRegionBytes = TN * 128;         // TN rows x 128 bytes
+  // K and V rings; a CTA stays under half an SM's shared memory.
   static constexpr int kKStages = D == 64 ? 3 : 2;
   static constexpr int kVStages = 2;
   static constexpr uint32_t kQOff = 0;
-  static constexpr uint32_t kKOff = kTileBytes;
-  static constexpr uint32_t kVOff = kKOff + kKStages * kTileBytes;
-  static constexpr uint32_t kBarOff = kVOff + kVStages * kTileBytes;
+  static constexpr uint32_t kKOff = kQBytes;
+  static constexpr uint32_t kVOff = kKOff + kKStages * kKVBytes;
+  static constexpr uint32_t kBarOff = kVOff + kVStages * kKVBytes;
   // q_full, k_full[KS], k_empty[KS], v_full[VS], v_empty[VS], s_full, s_free, p_full, o_done,
   // drain
   static constexpr int kNumBars = 1 + 2 * kKStages + 2 * kVStages + 5;
   static constexpr uint32_t kMiscOff = kBarOff + kNumBars * 8;
   static constexpr uint32_t kSmemBytes = kMiscOff + 16 + 1024;   // + alignment slack
-  static constexpr uint32_t kTmemS = 0;                 // S: 128 fp32 columns
-  static constexpr uint32_t kTmemP = 128;               // P: 64 columns of 16-bit pairs
-  static constexpr uint32_t kTmemO = D == 64 ? 192 : 256;
-  static constexpr uint32_t kTmemCols = D == 64 ? 256 : 512;
+  // TMEM, 256 columns so that two CTAs share an SM: S (TN fp32 columns) at
+  // 0, P (TN/2 columns of 16-bit pairs) at TN, O (D fp32 columns) at 256 - D.
+  // D = 64: S 0..127, P 128..191, O 192..255; D = 128: S 0..63, P 64..95,
+  // O 128..255.
+  static constexpr uint32_t kTmemS = 0;
+  static constexpr uint32_t kTmemP = TN;
+  static constexpr uint32_t kTmemO = 256 - D;
+  static constexpr uint32_t kTmemCols = 256;
+  static_assert(kTmemP + TN / 2 <= kTmemO, "TMEM layout overlaps");
 };
 
 struct Item {
@@ -97,9 +105,10 @@ __device__ __forceinline__ Item decode_item(const AttnParams& p) {
 }
 
 // Tile g of a stream's KV sequence -> (position in the visible table, tile in page, valid rows).
+template <int TN>
 __device__ __forceinline__ void tile_coords(const StreamPlan& sp, int P, int g, int& page_pos,
                                             int& t, int& valid) {
-  const int tpp = (P + kTileN - 1) / kTileN;
+  const int tpp = (P + TN - 1) / TN;
   const int full = (sp.n_pages - 1) * tpp;
   int page_tokens;
   if (g < full) {
@@ -111,7 +120,7 @@ __device__ __forceinline__ void tile_coords(const StreamPlan& sp, int P, int g, 
     t = g - full;
     page_tokens = sp.lpl;
   }
-  valid = min(kTileN, page_tokens - t * kTileN);
+  valid = min(TN, page_tokens - t * TN);
 }
 
 template <bool BF16>
@@ -126,7 +135,7 @@ __device__ __forceinline__ uint32_t pack2(float lo, float hi) {
 }
 
 template <int D, bool BF16>
-__global__ void __launch_bounds__(kThreads, D == 64 ? 2 : 1)
+__global__ void __launch_bounds__(kThreads, 2)
     attn_sm100_kernel(const __grid_constant__ CUtensorMap tmap_q,
                       const __grid_constant__ CUtensorMap tmap_kv,
                       const __grid_constant__ AttnParams p) {
@@ -152,6 +161,7 @@ __global__ void __launch_bounds__(kThreads, D == 64 ? 2 : 1)
   const uint32_t o_done = s_full + 24u;
   const uint32_t drain = s_full + 32u;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(gbase + C::kMiscOff);
+  constexpr int TN = C::TN;
   volatile int* abort_flag = reinterpret_cast<volatile int*>(gbase + C::kMiscOff + 4);
 
   const int warp = threadIdx.x / 32;
@@ -198,14 +208,14 @@ __global__ void __launch_bounds__(kThreads, D == 64 ? 2 : 1)
     if (lane == 0) {
       tma_prefetch_desc(&tmap_q);
       tma_prefetch_desc(&tmap_kv);
-      mbar_arrive_expect_tx(q_full, C::kTileBytes);
+      mbar_arrive_expect_tx(q_full, C::kQBytes);
       for (int r = 0; r < C::kRegions; ++r)
-        tma_load_3d(sQ + r * C::kRegionBytes, &tmap_q, q_full, r * 64, it.head,
+        tma_load_3d(sQ + r * C::kQRegionBytes, &tmap_q, q_full, r * 64, it.head,
                     sp.q_off + it.qtile * kTileM);
       int issued = 0, vissued = 0;
       for (int j = 0; j < n; ++j) {
         int page_pos, t, valid;
-        tile_coords(sp, p.P, it.t_begin + j, page_pos, t, valid);
+        tile_coords<TN>(sp, p.P, it.t_begin + j, page_pos, t, valid);
         int page = p.indices[sp.page_off + page_pos];
         if (page < 0 || page >= p.max_pages) {
           atomicOr(p.err, kErrPageId);
@@ -214,16 +224,16 @@ __global__ void __launch_bounds__(kThreads, D == 64 ? 2 : 1)
         const int c4 = (int)(p.block_page_base + page);
         const int sk = j % KS, sv = j % VS;
         if (!mbar_wait(k_empty(sk), ((j / KS) & 1) ^ 1, abort_flag, kWaitLimitNs)) { fail(); break; }
-        mbar_arrive_expect_tx(k_full(sk), C::kTileBytes);
+        mbar_arrive_expect_tx(k_full(sk), C::kKVBytes);
         for (int r = 0; r < C::kRegions; ++r)
-          tma_load_5d(sK + sk * C::kTileBytes + r * C::kRegionBytes, &tmap_kv, k_full(sk), r * 64,
-                      it.head, t * kTileN, 0, c4);
+          tma_load_5d(sK + sk * C::kKVBytes + r * C::kKVRegionBytes, &tmap_kv, k_full(sk), r * 64,
+                      it.head, t * TN, 0, c4);
         issued = j + 1;
         if (!mbar_wait(v_empty(sv), ((j / VS) & 1) ^ 1, abort_flag, kWaitLimitNs)) { fail(); break; }
-        mbar_arrive_expect_tx(v_full(sv), C::kTileBytes);
+        mbar_arrive_expect_tx(v_full(sv), C::kKVBytes);
         for (int r = 0; r < C::kRegions; ++r)
-          tma_load_5d(sV + sv * C::kTileBytes + r * C::kRegionBytes, &tmap_kv, v_full(sv), r * 64,
-                      it.head, t * kTileN, 1, c4);
+          tma_load_5d(sV + sv * C::kKVBytes + r * C::kKVRegionBytes, &tmap_kv, v_full(sv), r * 64,
+                      it.head, t * TN, 1, c4);
         vissued = j + 1;
       }
       if (*abort_flag) {
@@ -238,7 +248,7 @@ __global__ void __launch_bounds__(kThreads, D == 64 ? 2 : 1)
   } else if (warp == 5) {
     // ---------------------------------------------------------- MMA issuer
     if (lane == 0) {
-      constexpr uint32_t idS = idesc_f16(kTileM, kTileN, BF16, false);
+      constexpr uint32_t idS = idesc_f16(kTileM, TN, BF16, false);
       constexpr uint32_t idO = idesc_f16(kTileM, D, BF16, true);
       bool ok = mbar_wait(q_full, 0, abort_flag, kWaitLimitNs);
       tc_fence_after();
@@ -246,12 +256,13 @@ __global__ void __launch_bounds__(kThreads, D == 64 ? 2 : 1)
         const int s = j % KS;
         if (!mbar_wait(k_full(s), (j / KS) & 1, abort_flag, kWaitLimitNs)) return false;
         tc_fence_after();
-        const uint32_t kb = sK + s * C::kTileBytes;
+        const uint32_t kb = sK + s * C::kKVBytes;
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t off = (kk / 4) * C::kRegionBytes + (kk % 4) * 32;
-          mma_ss(tmem + C::kTmemS, desc_sw128(sQ + off, 16, 1024), desc_sw128(kb + off, 16, 1024),
-                 idS, kk > 0 ? 1u : 0u);
+          const uint32_t in_row = (kk % 4) * 32;
+          mma_ss(tmem + C::kTmemS, desc_sw128(sQ + (kk / 4) * C::kQRegionBytes + in_row, 16, 1024),
+                 desc_sw128(kb + (kk / 4) * C::kKVRegionBytes + in_row, 16, 1024), idS,
+                 kk > 0 ? 1u : 0u);
         }
         mma_commit(k_empty(s));
         mma_commit(s_full);
@@ -269,11 +280,11 @@ __global__ void __launch_bounds__(kThreads, D == 64 ? 2 : 1)
         if (!(ok = mbar_wait(p_full, j & 1, abort_flag, kWaitLimitNs))) break;
         if (!(ok = mbar_wait(v_full(s), (j / VS) & 1, abort_flag, kWaitLimitNs))) break;
         tc_fence_after();
-        const uint32_t vb = sV + s * C::kTileBytes;
+        const uint32_t vb = sV + s * C::kKVBytes;
 #pragma unroll
-        for (int kk = 0; kk < kTileN / 16; ++kk)
+        for (int kk = 0; kk < TN / 16; ++kk)
           mma_ts(tmem + C::kTmemO, tmem + C::kTmemP + kk * 8,
-                 desc_sw128(vb + kk * 2048, C::kRegionBytes, 1024), idO,
+                 desc_sw128(vb + kk * 2048, C::kKVRegionBytes, 1024), idO,
                  (j > 0 || kk > 0) ? 1u : 0u);
         mma_commit(v_empty(s));
         mma_commit(o_done);
@@ -302,12 +313,12 @@ __global__ void __launch_bounds__(kThreads, D == 64 ? 2 : 1)
     bool ok = true;
     // Position of the current tile in the visible table, advanced by one
     // tile per iteration (no divisions on the per-tile path).
-    const int tpp = (p.P + kTileN - 1) / kTileN;
+    const int tpp = (p.P + TN - 1) / TN;
     const int last_page = sp.n_pages - 1, lpl = sp.lpl, P = p.P;
     int page_pos, t, valid;
-    tile_coords(sp, P, it.t_begin, page_pos, t, valid);
+    tile_coords<TN>(sp, P, it.t_begin, page_pos, t, valid);
     for (int j = 0; j < n && ok; ++j) {
-      valid = min(kTileN, (page_pos < last_page ? P : lpl) - t * kTileN);
+      valid = min(TN, (page_pos < last_page ? P : lpl) - t * TN);
       if (++t == tpp && page_pos < last_page) {
         t = 0;
         ++page_pos;
@@ -315,27 +326,23 @@ __global__ void __launch_bounds__(kThreads, D == 64 ? 2 : 1)
       ok = __all_sync(kAll, mbar_wait(s_full, j & 1, abort_flag, kWaitLimitNs));
       if (!ok) break;
       tc_fence_after();
-      float s[128];
+      constexpr int NC = TN / 32;                     // 32-column chunks per tile
+      float s[TN];
       {
-        uint32_t r0[32], r1[32], r2[32], r3[32];
-        tmem_ld32(sb, r0);
-        tmem_ld32(sb + 32, r1);
-        tmem_ld32(sb + 64, r2);
-        tmem_ld32(sb + 96, r3);
+        uint32_t r[NC][32];
+#pragma unroll
+        for (int c = 0; c < NC; ++c) tmem_ld32(sb + 32 * c, r[c]);
         tmem_wait_ld();
         tc_fence_before();
         mbar_arrive(s_free);
 #pragma unroll
-        for (int i = 0; i < 32; ++i) {
-          s[i] = __uint_as_float(r0[i]);
-          s[32 + i] = __uint_as_float(r1[i]);
-          s[64 + i] = __uint_as_float(r2[i]);
-          s[96 + i] = __uint_as_float(r3[i]);
-        }
-      }
-      if (valid < kTileN) {
+        for (int c = 0; c < NC; ++c)
 #pragma unroll
-        for (int i = 0; i < 128; ++i) s[i] = i < valid ? s[i] : -INFINITY;
+          for (int i = 0; i < 32; ++i) s[32 * c + i] = __uint_as_float(r[c][i]);
+      }
+      if (valid < TN) {
+#pragma unroll
+        for (int i = 0; i < TN; ++i) s[i] = i < valid ? s[i] : -INFINITY;
       }
       // The exponentials are taken against the running maximum m of the
       // earlier tiles, without a reduction over this tile first.  P values
@@ -349,7 +356,7 @@ __global__ void __launch_bounds__(kThreads, D == 64 ? 2 : 1)
       {
         const float nm = -m;
 #pragma unroll
-        for (int c = 0; c < 4; ++c) {
+        for (int c = 0; c < NC; ++c) {
           uint32_t pk[16];
 #pragma unroll
           for (int i = 0; i < 16; ++i) {
@@ -381,7 +388,7 @@ __global__ void __launch_bounds__(kThreads, D == 64 ? 2 : 1)
 #pragma unroll
         for (int k = 0; k < 4; ++k) mm[k] = fmaxf(s[2 * k], s[2 * k + 1]);
 #pragma unroll
-        for (int i = 4; i < 64; ++i) mm[i % 4] = fmax3(mm[i % 4], s[2 * i], s[2 * i + 1]);
+        for (int i = 4; i < TN / 2; ++i) mm[i % 4] = fmax3(mm[i % 4], s[2 * i], s[2 * i + 1]);
         const float mx = fmaxf(fmaxf(mm[0], mm[1]), fmaxf(mm[2], mm[3])) * sl2;
         if (__any_sync(kAll, mx > m)) {
           // Recompute this tile against the new maximum and rescale the
@@ -397,7 +404,7 @@ __global__ void __launch_bounds__(kThreads, D == 64 ? 2 : 1)
           la[0] = la[1] = la[2] = la[3] = 0.f;
           tmem_wait_st();
 #pragma unroll
-          for (int c = 0; c < 4; ++c) {
+          for (int c = 0; c < NC; ++c) {
             uint32_t pk[16];
 #pragma unroll
             for (int i = 0; i < 16; ++i) {
@@ -511,7 +518,7 @@ int attn_items_per_stream(int H, int D, int qtiles, int chunks) {
   return H * qtiles * chunks;
 }
 
-int attn_ctas_per_sm(int D) { return D == 64 ? 2 : 1; }   // TMEM 256 and < 113 KB smem at D = 64
+int attn_ctas_per_sm(int D) { (void)D; return 2; }   // 256 TMEM columns and < 113 KB smem each
 
 cudaError_t launch_attn_sm100(const AttnParams& p, const void* tmap_q, const void* tmap_kv,
                               int dtype, cudaStream_t s) {

@@ -190,7 +190,7 @@ int encode_kv_map(svt_cache* c) {
   cuuint64_t strides[4] = {c->D * e, (cuuint64_t)c->H * c->D * e,
                            (cuuint64_t)c->P * c->H * c->D * e,
                            2ull * c->P * c->H * c->D * e};
-  cuuint32_t box[5] = {64, 1, (cuuint32_t)kTileN, 1, 1};
+  cuuint32_t box[5] = {64, 1, (cuuint32_t)attn_tile_n(c->D), 1, 1};
   cuuint32_t estr[5] = {1, 1, 1, 1, 1};
   CUresult r = enc(&c->tmap_kv,
                    c->dtype == SVT_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16
@@ -713,7 +713,8 @@ int svt_plan(svt_cache* c, const int32_t* qo_len, svt_stream_t) {
   if (!qo_len) return fail(SVT_EINVAL, "qo_len_per_stream is NULL");
   if (c->dirty) return fail(SVT_ESTATE, "cache changed since build_visible_page_table");
   const int P = c->P;
-  const int tpp = (P + kTileN - 1) / kTileN;
+  const int TN = attn_tile_n(c->D);
+  const int tpp = (P + TN - 1) / TN;
   int rows = 0, page_off = 0;
   AttnParams& a = c->attn;
   SimtParams& m = c->simt;
@@ -738,7 +739,7 @@ int svt_plan(svt_cache* c, const int32_t* qo_len, svt_stream_t) {
     sp.page_off = page_off;
     sp.n_pages = np;
     sp.lpl = lpl;
-    sp.tiles = np ? (np - 1) * tpp + (lpl + kTileN - 1) / kTileN : 0;
+    sp.tiles = np ? (np - 1) * tpp + (lpl + TN - 1) / TN : 0;
     tiles[i] = sp.tiles;
     qt[i] = sp.qtiles;
     rows += qo_len[i];
@@ -753,10 +754,10 @@ int svt_plan(svt_cache* c, const int32_t* qo_len, svt_stream_t) {
   for (int i = 0; i < c->n_streams; ++i)
     if (qo_len[i]) max_tiles = std::max(max_tiles, tiles[i]);
   // Cost model: a work item is one 128-row query tile over a KV chunk; a KV
-  // tile costs 4*128*128*D flops at 6.6 TFLOP/s per SM (a round figure near
+  // tile costs 4*128*TN*D flops at 6.6 TFLOP/s per SM (a round figure near
   // what the kernel sustains; only its ratio to the fixed per-item and merge
   // costs steers the choice), shared by the CTAs resident on one SM.
-  const double tile_us = 4.0 * kTileM * kTileN * c->D / 6.6e6 * attn_ctas_per_sm(c->D);
+  const double tile_us = 4.0 * kTileM * TN * c->D / 6.6e6 * attn_ctas_per_sm(c->D);
   const double item_us = 2.0;
   std::vector<int> best(c->n_streams, 1);
   double best_t = 1e300;

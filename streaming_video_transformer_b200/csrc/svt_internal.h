@@ -12,7 +12,10 @@ namespace svt {
 
 constexpr int kMaxSpecialSpan = 8;   // special pages one frame's specials can touch
 constexpr int kTileM = 128;          // query rows per tensor-core tile
-constexpr int kTileN = 128;          // KV tokens per tensor-core tile
+constexpr int kTileN = 128;          // KV tokens per tensor-core tile at D = 64
+// KV tokens per tile of the tensor-core attention kernel: 128 at D = 64, 64 at
+// D = 128, so that a CTA needs 256 TMEM columns and two CTAs share an SM.
+__host__ __device__ constexpr int attn_tile_n(int D) { return D == 64 ? kTileN : 64; }
 
 // Device error word bits (OR-ed by kernels, read by svt_device_error).
 enum : unsigned {
@@ -76,7 +79,7 @@ struct StreamPlan {
   int page_off;     // first entry of the stream in the visible table
   int n_pages;      // entries in the visible table
   int lpl;          // valid tokens on the last page
-  int tiles;        // KV tiles: (n_pages-1)*ceil(P/kTileN) + ceil(lpl/kTileN)
+  int tiles;        // KV tiles: (n_pages-1)*ceil(P/TN) + ceil(lpl/TN), TN = attn_tile_n(D)
   int item_off;     // first work item of the stream
 };
 

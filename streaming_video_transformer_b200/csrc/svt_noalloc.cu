@@ -110,7 +110,8 @@ extern "C" SVT_API int svt_attention_noalloc(
     return err(SVT_EINVAL, "q, out and pool_block must be 16-byte aligned");
 
   AttnParams a{};
-  const int tpp = (page_size + kTileN - 1) / kTileN;
+  const int TN = attn_tile_n(D);
+  const int tpp = (page_size + TN - 1) / TN;
   int rows = 0, qtiles_total = 0, min_tiles = 1 << 30;
   for (int i = 0; i < num_streams; ++i) {
     const int np = indptr[i + 1] - indptr[i];
@@ -125,7 +126,7 @@ extern "C" SVT_API int svt_attention_noalloc(
     if (qo_len[i] > 0) {
       if (np == 0) return err(SVT_EINVAL, "stream %d has queries but no pages", i);
       if (sp.lpl < 1 || sp.lpl > page_size) return err(SVT_EINVAL, "last_page_len out of range");
-      sp.tiles = (np - 1) * tpp + (sp.lpl + kTileN - 1) / kTileN;
+      sp.tiles = (np - 1) * tpp + (sp.lpl + TN - 1) / TN;
       min_tiles = std::min(min_tiles, sp.tiles);
     }
     rows += qo_len[i];
@@ -203,7 +204,7 @@ extern "C" SVT_API int svt_attention_noalloc(
                           (cuuint64_t)max_pages};
     cuuint64_t strides[4] = {(cuuint64_t)D * 2, (cuuint64_t)H * D * 2,
                              (cuuint64_t)page_size * H * D * 2, 2ull * page_size * H * D * 2};
-    cuuint32_t box[5] = {64, 1, (cuuint32_t)kTileN, 1, 1};
+    cuuint32_t box[5] = {64, 1, (cuuint32_t)attn_tile_n(D), 1, 1};
     cuuint32_t es[5] = {1, 1, 1, 1, 1};
     if (enc(&tkv, tdt, 5, const_cast<void*>(pool_block), dims, strides, box, es,
             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
