@@ -224,3 +224,36 @@ def test_set_free_lists_permutes_ids():
         c.set_free_lists(perm_p, perm_s)                    # not empty any more
     c.reset()
     assert c.get_cache_stats()["frame_count"] == 0
+
+
+@pytest.mark.parametrize("D,tile", [(64, 128), (128, 64)])
+def test_plan_tiles_items_and_split_bounds(D, tile):
+    """The plan's work decomposition: KV tiles per stream are whole pages of
+    ceil(page_size / tile) tiles plus ceil(last_page_len / tile) (the kernel
+    reads 128-token tiles at D = 64 and 64-token tiles at D = 128), one work
+    item per (head, 128-row query tile, KV chunk), and a chunk count between
+    1 and max_splits that never exceeds the stream's tile count."""
+    P, ns, S, W, H = 100, 6, 2, 3, 4
+    ages = (1, 4, 9)
+    qo = [P + ns, 2 * (P + ns), 5]
+    c = _host_cache(max_pages=3 * (S + W + 1) + 8, page_size=P, H=H, D=D, sliding_window=W,
+                    scale_frames=S, num_special=ns, num_streams=len(ages), max_splits=8,
+                    max_qo_len=sum(qo))
+    for s, age in enumerate(ages):
+        for _ in range(age):
+            c.append_frame(0, stream=s)
+            c.evict_frames(s)
+    c.build_visible_page_table()
+    c.plan(qo)
+    info = c.plan_info()
+    ip, ix, lp = c.get_page_table()
+    items = 0
+    for s, age in enumerate(ages):
+        n_pages = ip[s + 1] - ip[s]
+        tiles = (n_pages - 1) * -(-P // tile) + -(-int(lp[s]) // tile)
+        assert info["kv_tiles"][s] == tiles
+        assert info["kv_tokens"][s] == (n_pages - 1) * P + int(lp[s])
+        assert info["kv_tokens"][s] == min(age, S) * P + min(max(age - S, 0), W) * P + ns * age
+        assert 1 <= info["splits"][s] <= min(8, tiles)
+        items += H * -(-qo[s] // 128) * info["splits"][s]
+    assert info["num_items"] == items
