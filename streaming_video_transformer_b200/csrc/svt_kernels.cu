@@ -185,10 +185,12 @@ __global__ void __launch_bounds__(128) merge_kernel(AttnParams p) {
     if (row >= p.s[i].q_off && row < p.s[i].q_off + p.s[i].nq) chunks = p.s[i].chunks;
   if (chunks <= 1) return;                         // written directly by the attention kernel
   float mx = -INFINITY;
+#pragma unroll 4
   for (int c = 0; c < chunks; ++c)
     mx = fmaxf(mx, p.ws_lse[((size_t)c * p.ws_rows + row) * p.H + h]);
   float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
   float den = 0.f;
+#pragma unroll 4
   for (int c = 0; c < chunks; ++c) {
     const float w = __expf(p.ws_lse[((size_t)c * p.ws_rows + row) * p.H + h] - mx);
     const float4 o = reinterpret_cast<const float4*>(
@@ -197,11 +199,16 @@ __global__ void __launch_bounds__(128) merge_kernel(AttnParams p) {
     den += w;
   }
   const float inv = 1.f / den;
-  T* o = static_cast<T*>(p.out) + ((size_t)row * p.H + h) * p.D + lane * 4;
-  o[0] = from_f<T>(acc.x * inv);
-  o[1] = from_f<T>(acc.y * inv);
-  o[2] = from_f<T>(acc.z * inv);
-  o[3] = from_f<T>(acc.w * inv);
+  // four 16-bit outputs in one 8-byte store (D/4 lanes cover a row's head)
+  union {
+    T v[4];
+    uint2 u;
+  } pk;
+  pk.v[0] = from_f<T>(acc.x * inv);
+  pk.v[1] = from_f<T>(acc.y * inv);
+  pk.v[2] = from_f<T>(acc.z * inv);
+  pk.v[3] = from_f<T>(acc.w * inv);
+  *reinterpret_cast<uint2*>(static_cast<T*>(p.out) + ((size_t)row * p.H + h) * p.D + lane * 4) = pk.u;
   if (p.lse && lane == 0) p.lse[(size_t)row * p.H + h] = mx + logf(den);
 }
 
