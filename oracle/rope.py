@@ -2,7 +2,7 @@
 
 The pages say only that query and key are prepared with an optional RoPE
 before the key/value are appended ([P1] § Step-by-Step Streaming Inference,
-step 1).  The 2-D convention used here is a reading (listed in the design doc):
+step 1).  The 2-D convention used here is a reading of that silence:
 
   * patch p (0-based among the patch rows, raster order) sits at grid row
     r = p // grid and column c = p % grid; special rows are not rotated;

@@ -24,7 +24,7 @@ What it restates:
     special_tokens}``.  [P3] § Implementation Examples, "Inspecting Cache
     Statistics"; [P4] § Practical Usage Examples.
 
-Readings where the pages are silent (each also listed in the design doc):
+Readings where the pages are silent:
   * Input rows ``0..num_special-1`` of a frame are the special tokens and
     the remaining rows the patch tokens.
   * While a frame is provisional the window holds up to ``sliding_window+1``

@@ -1,7 +1,7 @@
 """Test-only model of the page allocator (predicts physical page ids).
 
 The pages fix the two-stream policy but not which physical page a frame
-gets.  The reading used (listed in the design doc): patch pages 0..patch_pages-1
+gets.  The reading used: patch pages 0..patch_pages-1
 and special pages patch_pages..max_pages-1 sit in two FIFO free lists handed
 out from the front; evicted window pages go to the back; a rolled-back frame
 returns its pages to the front.  This model restates that policy in plain

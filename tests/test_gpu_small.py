@@ -122,8 +122,9 @@ def test_edge_shapes(cfg):
     st = oracle_stream(w)
     # With RoPE the kernel rotates in fp32 (fused multiply-adds) and the
     # oracle in float64, each rounding once to the 16-bit storage type, so a
-    # rare rotated Q/K value differs by one storage step (the design's RoPE
-    # reading).  The fp32 path's bound is widened by twice the spread of the
+    # rare rotated Q/K value differs by one storage step (RoPE is taken as a
+    # rotation in fp32 rounded once to the storage type, so two valid
+    # roundings of it can disagree by one step).  The fp32 path's bound is widened by twice the spread of the
     # oracle run on the float64 rotation against a fused fp32 rotation, and
     # rotated keys in the pool are compared within one storage step.
     st32 = oracle_stream(w) if w.rope_grid else None
