@@ -37,9 +37,8 @@ def assert_close(gpu, ref, fp32=False, what="", fp32_tol=TOL_FP32_REL_L2):
 
 def rope2d_fused_fp32(x, num_special, grid, theta):
     """The 2-D RoPE rotation (patch row/column positions, rotate-half pairs)
-    evaluated in fp32, each output
-    one fused multiply-add over the other product rounded to fp32 (the way an
-    FMA unit evaluates a*c - b*s).  Like the float64 rotation it is a valid
+    evaluated in fp32, each output one fused multiply-add over the other
+    product rounded to fp32 (the way an FMA unit evaluates a*c - b*s).  Like the float64 rotation it is a valid
     evaluation of the same formula; rounded to a 16-bit storage type, the two
     can differ by one step on a rare element.  Tests use the spread between
     the oracle run on each to size the fp32 path's bound on RoPE workloads.

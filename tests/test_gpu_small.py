@@ -121,12 +121,12 @@ def test_edge_shapes(cfg):
     bank = FrameBank(w, 0, 0)
     st = oracle_stream(w)
     # With RoPE the kernel rotates in fp32 (fused multiply-adds) and the
-    # oracle in float64, each rounding once to the 16-bit storage type, so a
-    # rare rotated Q/K value differs by one storage step (RoPE is taken as a
-    # rotation in fp32 rounded once to the storage type, so two valid
-    # roundings of it can disagree by one step).  The fp32 path's bound is widened by twice the spread of the
-    # oracle run on the float64 rotation against a fused fp32 rotation, and
-    # rotated keys in the pool are compared within one storage step.
+    # oracle in float64, each rounding once to the 16-bit storage type: two
+    # valid roundings of the same rotation, which disagree by one storage
+    # step on a rare Q/K value.  The fp32 path's bound is widened by twice
+    # the spread of the oracle run on the float64 rotation against a fused
+    # fp32 rotation, and rotated keys in the pool are compared within one
+    # storage step.
     st32 = oracle_stream(w) if w.rope_grid else None
     for t in range(w.frames):
         q = _step(c, w, bank, t)
