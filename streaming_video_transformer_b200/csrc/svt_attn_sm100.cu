@@ -150,7 +150,7 @@ __global__ void __launch_bounds__(kThreads, 2)
   const uint32_t sV = base + C::kVOff;
   const uint32_t bars = base + C::kBarOff;
   const uint32_t q_full = bars;
-  constexpr int KS = C::kKStages, VS = C::kVStages;
+  constexpr int KS = C::kKStages, VS = C::kVStages, TN = C::TN;
   auto k_full = [&](int s) { return bars + 8u * (1 + s); };
   auto k_empty = [&](int s) { return bars + 8u * (1 + KS + s); };
   auto v_full = [&](int s) { return bars + 8u * (1 + 2 * KS + s); };
@@ -161,7 +161,6 @@ __global__ void __launch_bounds__(kThreads, 2)
   const uint32_t o_done = s_full + 24u;
   const uint32_t drain = s_full + 32u;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(gbase + C::kMiscOff);
-  constexpr int TN = C::TN;
   volatile int* abort_flag = reinterpret_cast<volatile int*>(gbase + C::kMiscOff + 4);
 
   const int warp = threadIdx.x / 32;
