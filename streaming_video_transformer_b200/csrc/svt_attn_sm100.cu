@@ -46,6 +46,13 @@ namespace {
 using namespace sm100;
 
 constexpr int kThreads = 192;
+// D = 64 launches 256 threads (two warpgroups) with 128 registers each and
+// moves registers from the producer/MMA warpgroup (warps 4-7, down to 64) to
+// the softmax warpgroup (warps 0-3, up to 192): 128 x 64 + 128 x 192 = 256 x
+// 128.  The build checks that the kernel's launch register count is 128; a
+// smaller count would leave the increase waiting for registers forever.
+constexpr int kSplitThreads = 256;
+constexpr int threads_for(int D) { return D == 64 ? kSplitThreads : kThreads; }
 constexpr uint64_t kWaitLimitNs = 2000000000ull;   // 2 s
 // A tile's P row is accepted while its sum stays at or below this bound, so
 // that every P value is at most 2^8 (within fp16's range for the P.V MMA).
@@ -135,7 +142,7 @@ __device__ __forceinline__ uint32_t pack2(float lo, float hi) {
 }
 
 template <int D, bool BF16>
-__global__ void __launch_bounds__(kThreads, 2)
+__global__ void __launch_bounds__(threads_for(D), 2)
     attn_sm100_kernel(const __grid_constant__ CUtensorMap tmap_q,
                       const __grid_constant__ CUtensorMap tmap_kv,
                       const __grid_constant__ AttnParams p) {
@@ -202,6 +209,8 @@ __global__ void __launch_bounds__(kThreads, 2)
     atomicOr(p.err, kErrWaitLimit);
   };
 
+  if (warp >= 4) {
+  if constexpr (D == 64) asm volatile("setmaxnreg.dec.sync.aligned.u32 64;\n" ::: "memory");
   if (warp == 4) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
@@ -293,7 +302,9 @@ __global__ void __launch_bounds__(kThreads, 2)
       mma_commit(drain);
       mbar_wait(drain, 0, nullptr, kWaitLimitNs);
     }
+  }
   } else {
+    if constexpr (D == 64) asm volatile("setmaxnreg.inc.sync.aligned.u32 192;\n" ::: "memory");
     // ------------------------------------------------------ softmax warps
     // Every tcgen05.ld/st runs on all 32 lanes of a warp (the branches around
     // them are warp-uniform).
@@ -357,12 +368,21 @@ __global__ void __launch_bounds__(kThreads, 2)
 #pragma unroll
         for (int c = 0; c < NC; ++c) {
           uint32_t pk[16];
+          if (c == NC - 1 && valid <= 32 * (NC - 1)) {
+            // The last chunk lies wholly past the tile's valid rows (the
+            // tail tile of a page): P = 0 without exponentiating -inf.
+            // Only the last chunk is tested, so no branch separates the
+            // exponentials of consecutive chunks.
 #pragma unroll
-          for (int i = 0; i < 16; ++i) {
-            const float p0 = ex2(fmaf(s[32 * c + 2 * i], sl2, nm));
-            const float p1 = ex2(fmaf(s[32 * c + 2 * i + 1], sl2, nm));
-            la[i % 4] += p0 + p1;
-            pk[i] = pack2<BF16>(p0, p1);
+            for (int i = 0; i < 16; ++i) pk[i] = 0u;
+          } else {
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+              const float p0 = ex2(fmaf(s[32 * c + 2 * i], sl2, nm));
+              const float p1 = ex2(fmaf(s[32 * c + 2 * i + 1], sl2, nm));
+              la[i % 4] += p0 + p1;
+              pk[i] = pack2<BF16>(p0, p1);
+            }
           }
           // P_{j-1}.V_{j-1} must have read the P columns (and finished
           // updating O) before P_j is written and O rescaled.  o_done is at
@@ -505,7 +525,7 @@ cudaError_t launch_t(const AttnParams& p, const void* tq, const void* tkv, cudaS
   CUtensorMap mq, mkv;
   memcpy(&mq, tq, sizeof(mq));
   memcpy(&mkv, tkv, sizeof(mkv));
-  kern<<<p.total_items, kThreads, C::kSmemBytes, s>>>(mq, mkv, p);
+  kern<<<p.total_items, threads_for(D), C::kSmemBytes, s>>>(mq, mkv, p);
   return cudaGetLastError();
 }
 
