@@ -41,10 +41,10 @@ SECONDARY = ("tiny_stream", "ragged4", "rollback10k")
 
 # DRAM traffic of one attention launch from the ncu capture summarised in
 # profiles/attn_sm100_vitl_step.md (single ViT-L step, 99,792 visible keys):
-# read 459.3 MB + write 24.4 MB.  Traffic grows with the visible keys, so the
+# read 461.1 MB + write 25.8 MB.  Traffic grows with the visible keys, so the
 # bench scales it to the mean key count of its timed frames.  Set to None when
 # the attention kernel changes until a new capture is taken.
-ATTN_TRAFFIC_BYTES, ATTN_TRAFFIC_KEYS = 483.62e6, 99792
+ATTN_TRAFFIC_BYTES, ATTN_TRAFFIC_KEYS = 486.82e6, 99792
 
 
 def _peaks():
