@@ -10,16 +10,18 @@
 // table, each full except the last (last_page_len valid tokens) -- with no
 // causal mask, read straight from the page pool.
 //
-// Work item = (stream, head, 128-row query tile, KV chunk); one CTA per item,
-// 192 threads; at D = 64 a CTA takes 256 TMEM columns and under half an SM's
-// shared memory, so two CTAs share an SM:
-//   warp 4      TMA producer: the Q tile once, then K and V tiles of 128
+// Work item = (stream, head, 128-row query tile, KV chunk); one CTA per item.
+// KV tiles hold TN tokens (128 at D = 64, 64 at D = 128), so a CTA takes 256
+// TMEM columns and under half an SM's shared memory and two CTAs share an SM.
+// D = 128 runs 192 threads; D = 64 runs 256 (warps 6-7 only hand their
+// registers to the softmax warpgroup):
+//   warp 4      TMA producer: the Q tile once, then K and V tiles of TN
 //               tokens gathered page by page through the visible table (a
-//               page is ceil(page_size/128) tiles; rows past the page end are
+//               page is ceil(page_size/TN) tiles; rows past the page end are
 //               zero-filled by TMA and masked).
 //   warp 5      MMA issuer (one thread) and TMEM owner:
-//                 S_j = Q K_j^T   (SS MMA, fp32 into TMEM columns 0..127)
-//                 O  += P_j V_j   (TS MMA: P_j from TMEM columns 128..191)
+//                 S_j = Q K_j^T   (SS MMA, fp32 into TMEM columns 0..TN-1)
+//                 O  += P_j V_j   (TS MMA: P_j from TMEM columns TN..3TN/2-1)
 //               S_{j+1} is issued as soon as the softmax has read S_j, so the
 //               tensor cores compute it while the softmax exponentiates S_j.
 //   warps 0-3   softmax: thread r owns query row r (TMEM lane r): reads S_j
