@@ -225,7 +225,8 @@ int encode_q_map(svt_cache* c, const void* q, int rows) {
 }
 
 void fill_rope_table(const svt_cache* c, std::vector<float2>& tab) {
-  // (cos, sin) of pos * theta^(-2i/m), m = D/2, i < m/2, pos < grid; double precision.
+  // (cos, sin) of pos * theta^(-2i/m), m = D/2, i < m/2, pos < grid: angle,
+  // cosine and sine in double precision, each value rounded once to fp32.
   const int m = c->D / 2, half = m / 2;
   tab.resize((size_t)c->rope_grid * half);
   for (int pos = 0; pos < c->rope_grid; ++pos)

@@ -31,6 +31,12 @@ template <> __device__ __forceinline__ float from_f<float>(float x) { return x; 
 // Rotates the 16-byte vectors `lo` (features i0..i0+VE-1 of a RoPE half) and
 // `hi` (features i0+m/2..) by angles of position `pos`:
 //   (a, b) -> (a cos - b sin, a sin + b cos),  angle_i = pos * theta^(-2i/m)
+// as one fixed fp32 computation, so that the rotated keys are reproducible
+// bit for bit: with c, s the fp32 table values,
+//   a' = rn(rn(a c) - rn(b s)),  b' = rn(rn(a s) + rn(b c)),
+// each operation rounded to nearest on its own (the _rn intrinsics keep the
+// compiler from contracting a product and a sum into one fused
+// multiply-add), then one rounding to the storage type.
 template <typename T>
 __device__ __forceinline__ void rope_pair(uint4& lo, uint4& hi, const float2* tab_row, int i0) {
   constexpr int VE = 16 / sizeof(T);
@@ -40,8 +46,8 @@ __device__ __forceinline__ void rope_pair(uint4& lo, uint4& hi, const float2* ta
   for (int j = 0; j < VE; ++j) {
     const float2 cs = tab_row[i0 + j];
     const float x = to_f(a[j]), y = to_f(b[j]);
-    a[j] = from_f<T>(fmaf(x, cs.x, -(y * cs.y)));
-    b[j] = from_f<T>(fmaf(x, cs.y, y * cs.x));
+    a[j] = from_f<T>(__fsub_rn(__fmul_rn(x, cs.x), __fmul_rn(y, cs.y)));
+    b[j] = from_f<T>(__fadd_rn(__fmul_rn(x, cs.y), __fmul_rn(y, cs.x)));
   }
 }
 

@@ -35,35 +35,6 @@ def assert_close(gpu, ref, fp32=False, what="", fp32_tol=TOL_FP32_REL_L2):
     return r
 
 
-def rope2d_fused_fp32(x, num_special, grid, theta):
-    """The 2-D RoPE rotation (patch row/column positions, rotate-half pairs)
-    evaluated in fp32, each output one fused multiply-add over the other
-    product rounded to fp32 (the way an FMA unit evaluates a*c - b*s).  Like the float64 rotation it is a valid
-    evaluation of the same formula; rounded to a 16-bit storage type, the two
-    can differ by one step on a rare element.  Tests use the spread between
-    the oracle run on each to size the fp32 path's bound on RoPE workloads.
-    Returns float64 [ns+grid*grid, H, D]."""
-    x = np.asarray(x.float().numpy() if hasattr(x, "float") else x, np.float32).copy()
-    D = x.shape[2]
-    m, half = D // 2, D // 4
-    inv_freq = theta ** (-2.0 * np.arange(half, dtype=np.float64) / m)
-    p = np.arange(grid * grid)
-    for sect, pos in ((0, p // grid), (1, p % grid)):
-        ang = pos[:, None].astype(np.float64) * inv_freq[None, :]
-        c = np.cos(ang).astype(np.float32)[:, None, :]
-        s = np.sin(ang).astype(np.float32)[:, None, :]
-        lo = slice(sect * m, sect * m + half)
-        hi = slice(sect * m + half, sect * m + m)
-        a = x[num_special:, :, lo].copy()
-        b = x[num_special:, :, hi].copy()
-        bs = (b * s).astype(np.float32).astype(np.float64)
-        bc = (b * c).astype(np.float32).astype(np.float64)
-        # a*c and a*s are exact in float64 (24 x 24 bits); one final rounding.
-        x[num_special:, :, lo] = (a.astype(np.float64) * c - bs).astype(np.float32)
-        x[num_special:, :, hi] = (a.astype(np.float64) * s + bc).astype(np.float32)
-    return x.astype(np.float64)
-
-
 def max_pages_for(w, frames_per_stream, num_streams=1, slack=2):
     """Patch pages S+W+1 per stream plus the special pages the streams need."""
     need_sp = sum(-(-f * w.ns // w.P) for f in frames_per_stream) + slack * num_streams

@@ -99,16 +99,10 @@ def test_vitl_stream24_blocks_0_and_23():
                 out = c.run(b, banks[b].device(t)[0])
                 ref, _ = oracle_out(sts[b], banks[b].oracle(t)[0], rows)
                 assert_close(out[rows], ref, what=f"block {b} t={t + 1}")
-    # RoPE'd keys in the pool: within one bf16 rounding step of the oracle's
+    # RoPE'd keys in the pool: the oracle's fp32 rotation, bit for bit
     gk, gv = gather_visible(c, 23, 0)
     ok, ov = sts[23].visible_kv()
-    assert np.array_equal(gv, ov)
-    # fp32 rotation vs float64 rotation, each rounded once to bf16: within one
-    # bf16 step of the value plus the fp32 arithmetic error of the rotation
-    # (a few 2^-24 of the input's magnitude, which dominates after cancellation).
-    diff = np.abs(gk - ok)
-    assert np.all(diff <= 2.0 ** -7 * np.abs(ok) + 4e-6)
-    assert np.mean(diff > 0) < 1e-3
+    assert np.array_equal(gk, ok) and np.array_equal(gv, ov)
     c.device_error()
 
 

@@ -243,14 +243,74 @@ def _rope_complex(x, ns, grid, theta):
 
 
 def test_rope_against_complex_form_and_identities():
+    """The fp32 rotation against the complex form in float64 on the same
+    (fp32) inputs: within the fp32 rounding of two products, their
+    difference and the tables (3 units of 2^-24 of |a| + |b|)."""
     rng = np.random.default_rng(9)
     ns, grid, theta = 3, 5, 100.0
-    x = rng.standard_normal((ns + grid * grid, 2, 16))
+    x = rng.standard_normal((ns + grid * grid, 2, 16)).astype(np.float32)
     y = rope2d(x, ns, grid, theta)
-    np.testing.assert_allclose(y, _rope_complex(x, ns, grid, theta), atol=1e-13)
+    assert y.dtype == np.float32
+    ref = _rope_complex(x, ns, grid, theta)
+    D = x.shape[2]; m = D // 2; half = m // 2
+    mag = np.empty_like(ref)
+    for base in (0, m):
+        pair = np.abs(x[..., base:base + half]) + np.abs(x[..., base + half:base + m])
+        mag[..., base:base + half] = pair
+        mag[..., base + half:base + m] = pair
+    assert np.all(np.abs(y - ref) <= 3.0 * 2.0 ** -24 * mag + 1e-30)
+    assert np.max(np.abs(y - ref)) > 0                            # rounding is not hidden
     np.testing.assert_array_equal(y[:ns], x[:ns])                 # specials untouched
-    np.testing.assert_allclose(y[ns], x[ns], atol=0)              # patch (0,0): identity
-    np.testing.assert_allclose(np.linalg.norm(y, axis=2), np.linalg.norm(x, axis=2), rtol=1e-13)
+    np.testing.assert_array_equal(y[ns], x[ns])                   # patch (0,0): identity, exact
+    np.testing.assert_allclose(np.linalg.norm(y.astype(np.float64), axis=2),
+                               np.linalg.norm(x.astype(np.float64), axis=2), rtol=1e-6)
+
+
+def test_rope_unit_vectors_give_fp32_tables_exactly():
+    """Rotating the unit vector of feature i returns, exactly, the fp32
+    rounding of cos and sin of pos * theta^(-2i/m) (Python's math library,
+    float64), with pos the patch's row in the first half and its column in
+    the second: rn(1*c) - rn(0*s) = c and rn(1*s) + rn(0*c) = s."""
+    import math
+    ns, grid, theta, D = 1, 4, 100.0, 16
+    m, half = D // 2, D // 4
+    for sect in (0, 1):
+        for i in range(half):
+            x = np.zeros((ns + grid * grid, 1, D), np.float32)
+            x[ns:, 0, sect * m + i] = 1.0
+            y = rope2d(x, ns, grid, theta)
+            for p in range(grid * grid):
+                pos = p // grid if sect == 0 else p % grid
+                ang = pos * theta ** (-2.0 * i / m)
+                assert y[ns + p, 0, sect * m + i] == np.float32(math.cos(ang))
+                assert y[ns + p, 0, sect * m + half + i] == np.float32(math.sin(ang))
+                others = np.delete(y[ns + p, 0], [sect * m + i, sect * m + half + i])
+                assert not np.any(others)
+
+
+def test_rope_fp32_and_float64_rotations_round_alike_to_bf16():
+    """Rounded to bf16, the fp32 rotation and the float64 one agree except
+    on elements whose float64 value lies within the fp32 error of a bf16
+    rounding boundary: there they differ by one bf16 step, or by the fp32
+    error itself where cancellation leaves a value far below |a| + |b|."""
+    rng = np.random.default_rng(11)
+    ns, grid, theta = 6, 37, 100.0
+    x = torch.randn((ns + grid * grid, 4, 64), generator=torch.Generator().manual_seed(11))
+    x = x.to(torch.bfloat16).float().numpy()
+    a = torch.from_numpy(rope2d(x, ns, grid, theta)).to(torch.bfloat16).double().numpy()
+    b = torch.from_numpy(_rope_complex(x, ns, grid, theta)).to(torch.bfloat16).double().numpy()
+    diff = a != b
+    assert np.mean(diff) < 1e-3
+    # one bf16 step of the value, or (after cancellation leaves a tiny value)
+    # the fp32 error of the rotation, 3 units of 2^-24 of the pair's |a|+|b|
+    D = x.shape[2]; m = D // 2; half = m // 2
+    mag = np.empty_like(x, dtype=np.float64)
+    for base in (0, m):
+        pair = np.abs(x[..., base:base + half]) + np.abs(x[..., base + half:base + m])
+        mag[..., base:base + half] = pair
+        mag[..., base + half:base + m] = pair
+    step = 2.0 ** (np.floor(np.log2(np.maximum(np.abs(b[diff]), 1e-30))) - 7)
+    assert np.all(np.abs(a[diff] - b[diff]) <= np.maximum(step * 1.0001, 4 * 2.0 ** -24 * mag[diff]))
 
 
 def test_rope_dot_product_depends_only_on_offset():
@@ -258,8 +318,9 @@ def test_rope_dot_product_depends_only_on_offset():
     ns, grid = 0, 6
     a = rng.standard_normal(16); b = rng.standard_normal(16)
     X = np.tile(a, (grid * grid, 1, 1)); Y = np.tile(b, (grid * grid, 1, 1))
-    RX, RY = rope2d(X, ns, grid, 100.0), rope2d(Y, ns, grid, 100.0)
+    RX = rope2d(X, ns, grid, 100.0).astype(np.float64)
+    RY = rope2d(Y, ns, grid, 100.0).astype(np.float64)
     for (r1, c1, r2, c2) in [(0, 0, 1, 2), (3, 3, 4, 5), (2, 1, 3, 3)]:
         d1 = RX[r1 * grid + c1, 0] @ RY[r2 * grid + c2, 0]
         d2 = RX[(r1 + 1) * grid + c1 - 0, 0] @ RY[(r2 + 1) * grid + c2, 0] if r2 + 1 < grid else d1
-        assert abs(d1 - d2) < 1e-12
+        assert abs(d1 - d2) < 1e-5
