@@ -254,6 +254,9 @@ SVT_API int svt_selftest_wait_limit(int limit_us, svt_stream_t s);
  * The first call on a device looks up the scratch array's device address (with that device
  * current); make it before any stream capture.  All calls share the scratch and calls that
  * overlap on the GPU race on it.
+ * A page id outside [0, max_pages) in `indices` is read as page 0 and a wait that hits its
+ * limit ends the work item early; both are recorded in a per-device error word that this
+ * call does not read (it does not synchronise): call svt_noalloc_device_error.
  * Errors: SVT_EINVAL (bad argument; num_splits whose partials exceed the 32 MiB scratch),
  * SVT_ECUDA. */
 SVT_API int svt_attention_noalloc(const void* q, void* out, float* lse, const void* pool_block,
@@ -261,6 +264,12 @@ SVT_API int svt_attention_noalloc(const void* q, void* out, float* lse, const vo
                                   const int32_t* last_page_len, const int32_t* qo_len,
                                   int num_streams, int max_pages, int page_size, int H, int D,
                                   int dtype, int num_splits, svt_stream_t s);
+
+/* Synchronises `s`, then reads and clears the current device's error word of
+ * svt_attention_noalloc (set by its kernels on a page id out of range or a wait that hit its
+ * limit, by every call since the last read).  Allocates nothing.  The paper has no
+ * counterpart.  Returns SVT_OK, SVT_EDEVICE (message in svt_last_error) or SVT_ECUDA. */
+SVT_API int svt_noalloc_device_error(svt_stream_t s);
 
 /* Message of the last failed call on this thread ("" if none). */
 SVT_API const char* svt_last_error(void);

@@ -23,7 +23,7 @@ EXPORTED = [
     "svt_execute_deferred_eviction", "svt_rollback_last_frame", "svt_build_visible_page_table",
     "svt_get_page_table", "svt_read_device_page_table", "svt_plan", "svt_get_plan_info",
     "svt_run", "svt_get_cache_stats", "svt_device_error", "svt_last_error",
-    "svt_attention_noalloc", "svt_selftest_wait_limit",
+    "svt_attention_noalloc", "svt_noalloc_device_error", "svt_selftest_wait_limit",
 ]
 
 
@@ -89,6 +89,7 @@ def load() -> ctypes.CDLL:
         "svt_last_error": (ctypes.c_char_p, []),
         "svt_attention_noalloc": (I, [VP, VP, VP, VP, VP, i32p, i32p, i32p, I, I, I, I, I, I, I,
                                       VP]),
+        "svt_noalloc_device_error": (I, [VP]),
         "svt_selftest_wait_limit": (I, [I, VP]),
     }
     for name, (res, args) in sig.items():

@@ -211,6 +211,12 @@ def attention_noalloc(q, out, pool_block, indices, indptr, last_page_len, qo_len
         dtype, num_splits, _stream_handle(cuda_stream)))
 
 
+def noalloc_device_error(cuda_stream=None) -> None:
+    """``svt_noalloc_device_error``: synchronises, reads and clears the device
+    error word of ``attention_noalloc``; raises SvtError(SVT_EDEVICE) if set."""
+    _check(L.load().svt_noalloc_device_error(_stream_handle(cuda_stream)))
+
+
 def selftest_wait_limit(limit_us: int, cuda_stream=None) -> None:
     """``svt_selftest_wait_limit``: raises SvtError(SVT_EDEVICE) when the bounded
     wait gave up at its limit, which is the expected outcome."""

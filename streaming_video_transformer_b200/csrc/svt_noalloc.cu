@@ -16,6 +16,11 @@
 // kernel writes every partial before the merge reads it, so nothing needs
 // clearing, but calls that overlap on the GPU (different streams, or other
 // host threads) race on it.
+//
+// The kernels report an out-of-range page id (they read page 0 instead) or a
+// wait that hit its limit in a device error word kept beside the scratch,
+// one per device.  svt_noalloc_device_error reads and clears it; until then
+// it keeps whatever the calls since the last read reported.
 
 #include <cuda.h>
 #include <cudaTypedefs.h>
@@ -112,7 +117,7 @@ extern "C" SVT_API int svt_attention_noalloc(
   AttnParams a{};
   const int TN = attn_tile_n(D);
   const int tpp = (page_size + TN - 1) / TN;
-  int rows = 0, qtiles_total = 0, min_tiles = 1 << 30;
+  int rows = 0, qtiles_total = 0;
   for (int i = 0; i < num_streams; ++i) {
     const int np = indptr[i + 1] - indptr[i];
     if (qo_len[i] < 0 || np < 0 || indptr[i] < 0) return err(SVT_EINVAL, "bad qo_len or indptr");
@@ -127,14 +132,14 @@ extern "C" SVT_API int svt_attention_noalloc(
       if (np == 0) return err(SVT_EINVAL, "stream %d has queries but no pages", i);
       if (sp.lpl < 1 || sp.lpl > page_size) return err(SVT_EINVAL, "last_page_len out of range");
       sp.tiles = (np - 1) * tpp + (sp.lpl + TN - 1) / TN;
-      min_tiles = std::min(min_tiles, sp.tiles);
     }
     rows += qo_len[i];
     qtiles_total += sp.qtiles;
   }
   if (rows == 0) return SVT_OK;
   // Split-KV chunks: enough work items for every resident CTA slot, capped
-  // by the scratch size and by the shortest stream.
+  // by the scratch size; a stream with fewer KV tiles than splits takes one
+  // chunk per tile (below).
   const size_t per_split = (size_t)rows * H * (D + 1);
   const int fit = (int)std::min<size_t>(64, kScratchFloats / per_split);
   int splits = num_splits;
@@ -155,7 +160,6 @@ extern "C" SVT_API int svt_attention_noalloc(
     splits = std::min({splits, fit, 16});
     splits = std::max(1, splits);
   }
-  splits = std::min(splits, std::max(1, min_tiles));
 
   float* scratch = nullptr;
   unsigned* err_word = nullptr;
@@ -218,5 +222,21 @@ extern "C" SVT_API int svt_attention_noalloc(
     e = launch_merge(a, dtype, s);
     if (e != cudaSuccess) return err(SVT_ECUDA, "merge launch: %s", cudaGetErrorString(e));
   }
+  return SVT_OK;
+}
+
+extern "C" SVT_API int svt_noalloc_device_error(svt_stream_t stream) {
+  float* scratch = nullptr;
+  unsigned* err_word = nullptr;
+  if (int r = setup_device(&scratch, &err_word)) return r;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  unsigned h = 0;
+  cudaError_t e = cudaMemcpyAsync(&h, err_word, sizeof(h), cudaMemcpyDeviceToHost, s);
+  if (e == cudaSuccess) e = cudaMemsetAsync(err_word, 0, sizeof(unsigned), s);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+  if (e != cudaSuccess) return err(SVT_ECUDA, "read no-alloc error word: %s", cudaGetErrorString(e));
+  if (h)
+    return err(SVT_EDEVICE, "device error 0x%x:%s%s", h, (h & kErrPageId) ? " page-id" : "",
+               (h & kErrWaitLimit) ? " wait-limit" : "");
   return SVT_OK;
 }
