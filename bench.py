@@ -39,11 +39,12 @@ PREFILL = {"vitl_stream24": 72, "vitl_step": 200}
 SECONDARY = ("tiny_stream", "ragged4", "rollback10k")
 
 
-# DRAM traffic of one attention launch from the ncu capture summarised in
-# profiles/attn_sm100_vitl_step.md (single ViT-L step, 99,792 visible keys):
-# read 461.1 MB + write 25.8 MB.  Traffic grows with the visible keys, so the
-# bench scales it to the mean key count of its timed frames.  Set to None when
-# the attention kernel changes until a new capture is taken.
+# DRAM traffic of one attention launch, from an ncu capture of the single
+# ViT-L step (one 1375-row frame over 99,792 visible keys, 5 KV splits):
+# dram__bytes_read.sum 461.1 MB + dram__bytes_write.sum 25.8 MB.  Traffic
+# grows with the visible keys, so the bench scales it to the mean key count of
+# its timed frames.  Set to None when the attention kernel changes until a new
+# capture is taken.
 ATTN_TRAFFIC_BYTES, ATTN_TRAFFIC_KEYS = 486.82e6, 99792
 
 
@@ -249,46 +250,68 @@ def run_gpu(args, rank, world, local_rank):
     flops_per_block = [4.0 * w.Nq * _visible(t + 1, w) * w.H * w.D for t in timed_frames]
     total_flops = L * sum(flops_per_block)
 
-    # --- end-to-end: inputs copied from pinned host memory every frame -------
-    copy_stream = torch.cuda.Stream(device=dev)
+    # --- end-to-end: every frame's Q/K/V of all blocks copied in from pinned
+    # host memory, and every block's output copied back to pinned host memory.
+    # Copies in and out run on their own streams, double-buffered by frame
+    # parity, so they overlap the attention of the neighbouring frames.
+    h2d_stream = torch.cuda.Stream(device=dev)
+    d2h_stream = torch.cuda.Stream(device=dev)
     stage = [[[torch.empty_like(x) for x in devin[b][0]] for b in range(L)] for _ in range(2)]
-    copied = [torch.cuda.Event() for _ in range(2)]
-    consumed = [torch.cuda.Event() for _ in range(2)]
-    res_host = torch.empty((w.Nq, w.H, w.D), dtype=torch.bfloat16).pin_memory()
+    outs = [[torch.empty((w.Nq, w.H, w.D), dtype=torch.bfloat16, device=dev) for _ in range(L)]
+            for _ in range(2)]
+    res_host = [[torch.empty((w.Nq, w.H, w.D), dtype=torch.bfloat16).pin_memory()
+                 for _ in range(L)] for _ in range(2)]
+    copied = [torch.cuda.Event() for _ in range(2)]       # inputs of a parity landed
+    consumed = [torch.cuda.Event() for _ in range(2)]     # inputs of a parity used
+    computed = [torch.cuda.Event() for _ in range(2)]     # outputs of a parity written
+    drained = [torch.cuda.Event() for _ in range(2)]      # outputs of a parity copied out
     e_start, e_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    h2d = 0
+    h2d = d2h = 0
 
-    def enqueue_copy(i, t):
+    def enqueue_copy_in(i, t):
         nonlocal h2d
-        with torch.cuda.stream(copy_stream):
-            copy_stream.wait_event(consumed[i % 2])
+        with torch.cuda.stream(h2d_stream):
+            h2d_stream.wait_event(consumed[i % 2])
             for b in range(L):
                 for dst, src in zip(stage[i % 2][b], host[b][t % w.R]):
                     dst.copy_(src, non_blocking=True)
                     h2d += src.numel() * src.element_size()
-            copied[i % 2].record(copy_stream)
+            copied[i % 2].record(h2d_stream)
 
-    for ev in consumed:
+    def enqueue_copy_out(i):
+        nonlocal d2h
+        with torch.cuda.stream(d2h_stream):
+            d2h_stream.wait_event(computed[i % 2])
+            for b in range(L):
+                res_host[i % 2][b].copy_(outs[i % 2][b], non_blocking=True)
+                d2h += outs[i % 2][b].numel() * outs[i % 2][b].element_size()
+            drained[i % 2].record(d2h_stream)
+
+    for ev in consumed + drained:
         ev.record(stream)
     barrier()
     torch.cuda.synchronize()
     t0 = t_frame
     e_start.record(stream)
-    enqueue_copy(0, t0)
+    enqueue_copy_in(0, t0)
     for i in range(e2e_steps):
         if i + 1 < e2e_steps:
-            enqueue_copy(i + 1, t0 + i + 1)
+            enqueue_copy_in(i + 1, t0 + i + 1)
         stream.wait_event(copied[i % 2])
+        stream.wait_event(drained[i % 2])
         buf = stage[i % 2]
-        step(t0 + i, lambda b, t: buf[b])
+        step(t0 + i, lambda b, t: buf[b], outs=outs[i % 2])
         consumed[i % 2].record(stream)
-        res_host.copy_(out, non_blocking=True)            # the frame's result (last block)
+        computed[i % 2].record(stream)
+        enqueue_copy_out(i)
+    for ev in drained:
+        stream.wait_event(ev)
     e_end.record(stream)
     torch.cuda.synchronize()
     barrier()
     e2e_ms = e_start.elapsed_time(e_end)
     h2d_per_step = h2d // e2e_steps
-    d2h_per_step = res_host.numel() * res_host.element_size()
+    d2h_per_step = d2h // e2e_steps
     e2e_flops = L * sum(4.0 * w.Nq * _visible(t0 + i + 1, w) * w.H * w.D for i in range(e2e_steps))
 
     elapsed_ms, e2e_ms = max_over_ranks([elapsed_ms, e2e_ms], world, dev)
@@ -461,6 +484,47 @@ def cpu_threads():
         return os.cpu_count() or 1
 
 
+def cpu_model():
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except Exception:
+        pass
+    return "unknown"
+
+
+def oracle_vitl_step_one_thread_seconds():
+    """The oracle on the single ViT-L step (cache pre-filled with 200 frames,
+    one 1375-row frame attends over 99,768 tokens) with its BLAS limited to
+    one thread.  One head of the sixteen is timed (gather of that head's
+    visible K/V and its attention); the step time is 16 x that."""
+    import torch
+    from threadpoolctl import threadpool_limits
+
+    from oracle import FrameStream, attend
+    from streaming_video_transformer_b200.inputs import WORKLOADS, frame_qkv
+
+    w = WORKLOADS["vitl_step"]
+    data = [tuple(x.double().numpy() for x in frame_qkv(w, 0, 0, i)) for i in range(w.R)]
+    st = FrameStream(w.P, w.ns, w.S, w.W)
+    for t in range(w.frames):
+        st.append_frame(data[t % w.R][1], data[t % w.R][2])
+    q = data[(w.frames - 1) % w.R][0]
+    with threadpool_limits(limits=1), torch.autograd.no_grad():
+        torch_threads = torch.get_num_threads()
+        torch.set_num_threads(1)
+        try:
+            t0 = time.perf_counter()
+            k, v = st.visible_kv(heads=slice(0, 1))
+            attend(q[:, 0:1], k, v)
+            secs = time.perf_counter() - t0
+        finally:
+            torch.set_num_threads(torch_threads)
+    return w.H * secs, st.num_visible_tokens()
+
+
 def run_reference(args):
     """The CPU oracle as it stands, on the same workload: each step streams
     one frame into the oracle's cache and computes attention for a sample of
@@ -592,10 +656,16 @@ def main():
         try:
             secs = oracle_block_frame_seconds(w, r["last_timed"])
             cpu = {"value": 1.0 / (w.blocks * secs), "unit": "frames/s", "cores": cpu_threads(),
-                   "kind": "oracle",
+                   "kind": "oracle", "cpu_model": cpu_model(),
                    "sample": f"one of 24 blocks at frame t={r['last_timed']} (all 1375 query rows, "
                              f"16 heads, {_visible(r['last_timed'], w)} visible tokens); "
                              f"{secs:.1f} s x 24 blocks per frame"}
+            s1, nk = oracle_vitl_step_one_thread_seconds()
+            cpu["one_thread_vitl_step"] = {
+                "seconds_per_step": s1, "cores": 1,
+                "tflops": 4.0 * 1375 * nk * 16 * 64 / s1 / 1e12,
+                "sample": f"single ViT-L step (1375 query rows over {nk} visible tokens), BLAS "
+                          f"limited to one thread; one head of 16 timed, x16"}
         except Exception as exc:  # the CPU leg never blocks the GPU number
             cpu = {"value": None, "unit": "frames/s", "cores": cpu_threads(), "kind": "oracle",
                    "sample": f"failed: {exc!r}"}
@@ -613,17 +683,19 @@ def main():
         "tflops": tflops,
         "tflops_frac_of_peak": {"burst": tflops / burst, "sustained": tflops / sustained,
                                 "peak_kind": peak_kind},
-        "roofline": {"bound": "tensor", "achieved": achieved, "peak": sustained,
-                     "unit": "TFLOP/s", "frac": achieved / sustained, "traffic": traffic,
+        "roofline": {"bound": "tensor", "achieved": achieved, "peak": burst,
+                     "unit": "TFLOP/s", "frac": achieved / burst, "traffic": traffic,
                      "kernel": "svt_run (RoPE on Q + tcgen05 attention + split merge), block 0 "
                                "of every timed frame, CUDA events on the launch stream",
-                     "peak_kind": f"bf16 sustained ({peak_kind})",
-                     "frac_of_burst": achieved / burst},
+                     "peak_kind": f"dense bf16 burst ({peak_kind}): each launch is timed on its "
+                                  f"own at the running clock",
+                     "frac_of_sustained": achieved / sustained},
         "cpu_baseline": cpu,
         "e2e": {"value": e2e_fps, "unit": "frames/s", "h2d_bytes_per_step": r["h2d_per_step"],
                 "d2h_bytes_per_step": r["d2h_per_step"], "steps": r["e2e_steps"],
-                "note": f"inputs of all {w.blocks} blocks copied from pinned host memory each frame on "
-                        "a copy stream (double-buffered), last block's output read back"},
+                "note": f"Q/K/V of all {w.blocks} blocks copied from pinned host memory and the "
+                        f"outputs of all {w.blocks} blocks copied back to pinned host memory every "
+                        "frame, on two copy streams (double-buffered by frame parity)"},
         "gpu_launches": r["kernels_per_step"] * args.steps,
         "clocks": r["clocks"],
     }
