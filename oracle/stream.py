@@ -34,6 +34,15 @@ Readings where the pages are silent:
   * The visible order is scale frames' patches, then window patches oldest
     to newest, then all special tokens in frame order ([P4] FAQ "How does the
     paged cache handle variable sequence lengths": scale -> live -> special).
+  * ``cross_frame_special=False`` ([P3] § Configuration Parameters: the flag
+    retains the special tokens of evicted frames; [P3] § Sliding-Window
+    Eviction Strategy, "Special Token Retention"): without retention a
+    frame's special tokens are visible exactly while its patch tokens are,
+    i.e. for the scale frames and the window frames.  Each visible frame then
+    contributes its patch tokens followed by its special tokens, scale frames
+    first, window frames oldest to newest ([P3] § The Paged KV-Cache
+    Architecture: append_frame places patch tokens first, then special
+    tokens).
 """
 
 from __future__ import annotations
@@ -44,7 +53,7 @@ from ._util import as64
 
 
 def visible_frame_ids(n_frames: int, scale_frames: int, sliding_window: int,
-                      provisional: bool):
+                      provisional: bool, cross_frame_special: bool = True):
     """Frame indices whose tokens are visible after the current step.
 
     Returns ``(scale_ids, window_ids, special_ids)`` for a stream holding
@@ -55,15 +64,20 @@ def visible_frame_ids(n_frames: int, scale_frames: int, sliding_window: int,
     rest = list(range(S, n)) if n > S else []
     w = W + (1 if provisional else 0)
     window_ids = rest[len(rest) - w:] if 0 < w < len(rest) else (rest if w > 0 else [])
-    special_ids = list(range(n))
+    special_ids = list(range(n)) if cross_frame_special else scale_ids + window_ids
     return scale_ids, window_ids, special_ids
 
 
-def visible_token_count(n_frames, P, ns, S, W, provisional=False) -> int:
-    """min(t,S)*P + min(max(t-S,0), W[+1])*P + ns*t."""
+def visible_token_count(n_frames, P, ns, S, W, provisional=False,
+                        cross_frame_special=True) -> int:
+    """min(t,S)*P + min(max(t-S,0), W[+1])*P + ns*t, or, without cross-frame
+    special retention, (min(t,S) + min(max(t-S,0), W[+1]))*(P+ns)."""
     t = int(n_frames)
     w = W + (1 if provisional else 0)
-    return min(t, S) * P + min(max(t - S, 0), w) * P + ns * t
+    frames = min(t, S) + min(max(t - S, 0), w)
+    if not cross_frame_special:
+        return frames * (P + ns)
+    return frames * P + ns * t
 
 
 class _Frame:
@@ -82,11 +96,12 @@ class FrameStream:
     """One stream of one transformer block: per-frame K/V in Python lists."""
 
     def __init__(self, patches_per_frame: int, num_special: int,
-                 scale_frames: int, sliding_window: int):
+                 scale_frames: int, sliding_window: int, cross_frame_special: bool = True):
         self.P = int(patches_per_frame)
         self.ns = int(num_special)
         self.S = int(scale_frames)
         self.W = int(sliding_window)
+        self.cross_frame_special = bool(cross_frame_special)
         self.frames: list[_Frame] = []
         self.provisional = False
 
@@ -118,8 +133,9 @@ class FrameStream:
         self.provisional = False
 
     def _evict(self) -> None:
-        # Frames that left the window never come back: drop their patch data
-        # (keeps the oracle's memory bounded on long streams).
+        # Frames that left the window never come back: drop their patch data,
+        # and their special data without cross-frame retention (keeps the
+        # oracle's memory bounded on long streams).
         _, window, _ = visible_frame_ids(len(self.frames), self.S, self.W, False)
         first_live = window[0] if window else len(self.frames)
         for i in range(self.S, first_live):
@@ -127,10 +143,13 @@ class FrameStream:
             if f.k_patch is None:
                 continue
             f.k_patch = f.v_patch = None
+            if not self.cross_frame_special:
+                f.k_special = f.v_special = None
 
     # -- queries --------------------------------------------------------
     def visible_ids(self):
-        return visible_frame_ids(len(self.frames), self.S, self.W, self.provisional)
+        return visible_frame_ids(len(self.frames), self.S, self.W, self.provisional,
+                                 self.cross_frame_special)
 
     def visible_kv(self, heads=None):
         """(K, V) of all visible tokens, ``[N, H, D]`` float64, in the order
@@ -144,14 +163,18 @@ class FrameStream:
             assert f.k_patch is not None, "visible frame lost its patches"
             ks.append(f.k_patch[:, sel])
             vs.append(f.v_patch[:, sel])
-        for i in special:
-            ks.append(self.frames[i].k_special[:, sel])
-            vs.append(self.frames[i].v_special[:, sel])
+            if not self.cross_frame_special:       # the frame's own specials follow
+                ks.append(f.k_special[:, sel])
+                vs.append(f.v_special[:, sel])
+        if self.cross_frame_special:
+            for i in special:
+                ks.append(self.frames[i].k_special[:, sel])
+                vs.append(self.frames[i].v_special[:, sel])
         return np.concatenate(ks, 0), np.concatenate(vs, 0)
 
     def num_visible_tokens(self) -> int:
         return visible_token_count(len(self.frames), self.P, self.ns, self.S,
-                                   self.W, self.provisional)
+                                   self.W, self.provisional, self.cross_frame_special)
 
     def stats(self, patch_capacity: int) -> dict:
         """Cache statistics of this stream when the pool holds

@@ -21,15 +21,20 @@ def _eval_e(expr):
     return eval(expr, {"__builtins__": {}}, {"e": math.e})
 
 
-def two_frame_cases():
+def two_frame_cases(cross_frame_special=True):
+    """Cases and page tables of the two-frame example, with (default) or
+    without cross-frame special retention."""
+    case_tag, table_tag = ("case", "table") if cross_frame_special else ("nocross",
+                                                                          "table_nocross")
     cases, tables = [], []
     for line in _lines("two_frame_example.txt"):
         head, _, vals = line.partition(":")
+        tag = head.split()[0]
         kv = dict(tok.split("=") for tok in head.split()[1:])
-        if line.startswith("case"):
+        if tag == case_tag:
             cases.append((int(kv["S"]), int(kv["W"]), int(kv["t"]), int(kv["row"]),
                           [_eval_e(x) for x in vals.split(",")]))
-        elif line.startswith("table"):
+        elif tag == table_tag:
             body = dict(tok.split("=") for tok in vals.split())
             tables.append((int(kv["S"]), int(kv["W"]), int(kv["t"]),
                            body["indices"].split(","), int(body["last_page_len"])))

@@ -42,6 +42,21 @@ def test_two_frame_hand_example():
                                    err_msg=f"S={S} W={W} t={t} row={row}")
 
 
+def test_two_frame_hand_example_without_cross_frame_special():
+    cases, _ = golden_io.two_frame_cases(cross_frame_special=False)
+    assert len(cases) == 7
+    q, f0, f1 = _two_frame_inputs()
+    for S, W, t, row, expected in cases:
+        st = FrameStream(patches_per_frame=2, num_special=1, scale_frames=S, sliding_window=W,
+                         cross_frame_special=False)
+        for f in (f0, f1)[:t]:
+            st.append_frame(*f)
+        k, v = st.visible_kv()
+        o = attend(q, k, v)
+        np.testing.assert_allclose(o[row, 0], expected, rtol=0, atol=1e-14,
+                                   err_msg=f"no retention S={S} W={W} t={t} row={row}")
+
+
 def test_cache_stats_example_from_pages():
     g = golden_io.kv_file("cache_stats_example.txt")
     st = FrameStream(patches_per_frame=3, num_special=g["num_special"],
@@ -63,6 +78,12 @@ def test_visible_counts_golden():
         st.append_frame(x, x)
         assert st.num_visible_tokens() == counts[t - 1]
         assert st.visible_kv()[0].shape[0] == counts[t - 1]
+    counts_nc = [int(x) for x in vc["tiny_nocross"][1]]
+    st_nc = FrameStream(16, 6, 2, 4, cross_frame_special=False)
+    for t in range(1, 13):
+        st_nc.append_frame(x, x)
+        assert st_nc.num_visible_tokens() == counts_nc[t - 1]
+        assert st_nc.visible_kv()[0].shape[0] == counts_nc[t - 1]
     # special pages / last page length of the tiny stream at t=12
     body = dict(tok.split("=") for tok in vc["tiny_pages"][1])
     n_sp = 6 * 12
@@ -109,11 +130,14 @@ def _fifo_visibility(events, S, W):
     return set(scale) | set(window), frames
 
 
+@pytest.mark.parametrize("cross", [True, False])
 @pytest.mark.parametrize("S,W,seed", [(2, 4, 0), (0, 3, 1), (3, 1, 2), (1, 0, 3), (4, 2, 4)])
-def test_bruteforce_masked_attention(S, W, seed):
+def test_bruteforce_masked_attention(S, W, seed, cross):
+    """Without cross-frame special retention a special token's mask entry is
+    its frame's patch visibility; with it, 0 always."""
     rng = np.random.default_rng(seed)
     P, ns, H, D = 5, 2, 2, 8
-    st = FrameStream(P, ns, S, W)
+    st = FrameStream(P, ns, S, W, cross_frame_special=cross)
     all_k, all_v, events, store = {}, {}, [], {}
     fid = 0
     for step in range(11):
@@ -140,7 +164,8 @@ def test_bruteforce_masked_attention(S, W, seed):
             for r in range(ns + P):
                 is_special = r < ns
                 ks.append(k_f[r]); vs.append(v_f[r])
-                mask.append(0.0 if (is_special or f in vis_patch) else -np.inf)
+                visible = (is_special and cross) or f in vis_patch
+                mask.append(0.0 if visible else -np.inf)
         K = torch.tensor(np.stack(ks)).permute(1, 0, 2)         # [H,N,D]
         V = torch.tensor(np.stack(vs)).permute(1, 0, 2)
         q = rng.standard_normal((ns + P, H, D))
@@ -191,17 +216,19 @@ def test_lse_matches_logsumexp_and_sdpa():
 
 
 # --------------------------------------------------------------- invariants
-def test_visible_count_formula_on_random_streams():
+@pytest.mark.parametrize("cross", [True, False])
+def test_visible_count_formula_on_random_streams(cross):
     rng = np.random.default_rng(8)
     for _ in range(20):
         P, ns = int(rng.integers(1, 6)), int(rng.integers(0, 4))
         S, W = int(rng.integers(0, 4)), int(rng.integers(0, 5))
-        st = FrameStream(P, ns, S, W)
+        st = FrameStream(P, ns, S, W, cross_frame_special=cross)
         x = np.zeros((ns + P, 1, 4))
         for t in range(1, 15):
             deferred = rng.random() < 0.3
             st.append_frame(x, x, deferred=deferred)
-            expect = min(t, S) * P + min(max(t - S, 0), W + (1 if deferred else 0)) * P + ns * t
+            frames = min(t, S) + min(max(t - S, 0), W + (1 if deferred else 0))
+            expect = frames * P + ns * t if cross else frames * (P + ns)
             if ns + P and expect:
                 assert st.visible_kv()[0].shape[0] == expect
             if deferred:
