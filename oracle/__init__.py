@@ -16,12 +16,16 @@ Sources (web pages on the LingBot-Map streaming scheme, cited by title):
   [P3] "How LingBot-Map Uses KV Caching for Efficient Streaming Inference"
   [P4] "How FlashInfer's Paged KV Cache Attention Outperforms SDPA Fallback in Streaming Inference"
 
-Pins (tests/test_oracle_*.py): the hand-worked two-frame example
-(tests/golden/two_frame_example.txt), the cache-statistics example printed in
-[P3] and [P4] (tests/golden/cache_stats_example.txt), brute-force attention
-with an explicit visibility mask, torch's float64 scaled-dot-product
-attention, closed-form special cases (uniform and one-hot attention), the
-visible-token-count formula, rollback restoring outputs, and RoPE identities.
+Pins (tests/test_oracle.py): the hand-worked two-frame example, with and
+without cross-frame special retention (tests/golden/two_frame_example.txt),
+the cache-statistics example printed in [P3] and [P4]
+(tests/golden/cache_stats_example.txt), visible-token counts
+(tests/golden/visible_counts.txt), brute-force attention with an explicit
+visibility mask, torch's float64 scaled-dot-product attention, closed-form
+special cases (uniform and one-hot attention), the visible-token-count
+formula, rollback restoring outputs, and the RoPE rotation against a complex
+form within its fp32 error bound, with unit vectors giving the fp32 tables
+exactly.
 """
 
 from .stream import FrameStream, visible_frame_ids
