@@ -80,8 +80,19 @@ typedef struct svt_cache_opts {
   int host_only;     /* 1: bookkeeping only -- no device memory, no kernels; k/v/q must be NULL
                         and device calls return SVT_EINVAL.  For hosts without a GPU. */
   void* pool;        /* device memory of svt_pool_bytes() bytes, 256-byte aligned, owned by
-                        the caller; laid out [num_blocks][max_pages][2 (K,V)][page_size][H][D].
+                        the caller; laid out [num_blocks][max_pages][2 (K,V)][page_tokens][H][D]
+                        with page_tokens = page_size, or page_size + num_special when
+                        no_cross_frame_special is set.
                         Required unless host_only.  [P4] Sec. Physical Memory Layout. */
+  int no_cross_frame_special;
+                     /* 0 (default): the special tokens of every frame stay visible for good
+                        (kv_cache_cross_frame_special = True).  1: they leave with their frame's
+                        patch tokens (kv_cache_cross_frame_special = False, [P3] Sec.
+                        Configuration Parameters; Sec. Sliding-Window Eviction Strategy, "Special
+                        Token Retention").  Each frame then has one page of page_size +
+                        num_special tokens, its patch rows followed by its special rows ([P3]
+                        Sec. The Paged KV-Cache Architecture); no special pages are used,
+                        max_pages may equal patch_pages, and every visible page is full. */
 } svt_cache_opts;
 
 typedef struct svt_stats {
@@ -103,7 +114,8 @@ typedef struct svt_plan_info {
 /* Fills *opts with the defaults above (sizes that depend on the cache shape are 0 = derive). */
 SVT_API void svt_default_opts(svt_cache_opts* opts);
 
-/* Bytes of the caller-allocated pool: num_blocks*max_pages*2*page_size*H*D*sizeof(dtype).
+/* Bytes of the caller-allocated pool: num_blocks*max_pages*2*page_tokens*H*D*sizeof(dtype),
+ * page_tokens = page_size (+ num_special with no_cross_frame_special).
  * Returns 0 on invalid arguments.  [P2] Sec. Physical Memory Layout; [P4] Sec. Physical
  * Memory Layout (dimension 1 separates keys and values). */
 SVT_API size_t svt_pool_bytes(int max_pages, int page_size, int H, int D, const svt_cache_opts* opts);
@@ -221,6 +233,27 @@ SVT_API int svt_get_plan_info(const svt_cache* c, svt_plan_info* out);
  * planned stream), SVT_EINVAL, SVT_ECUDA. */
 SVT_API int svt_run(svt_cache* c, int block, const void* q, void* out, float* lse, int force_fp32,
             svt_stream_t s);
+
+/* One whole frame step of one stream, from a single call: for every block b the frame's
+ * k[b], v[b] are appended (svt_append_frame), then svt_evict_frames, svt_build_visible_page_table
+ * and svt_plan (query rows = the frame's num_special + page_size rows on `stream`, none on the
+ * others) run, then svt_run(b, q[b], out[b], lse = NULL, force_fp32 = 0) for every block.
+ * k, v, q, out: HOST arrays of num_blocks DEVICE pointers.  Deferred eviction applies as set by
+ * svt_set_defer_eviction.  [P1] Sec. Step-by-Step Streaming Inference; [P1] Sec. Implementation
+ * Examples (the upstream captures a block's forward in a CUDA graph).
+ * use_graph = 0: the kernels are launched one by one, as by the separate calls.
+ * use_graph = 1: the step's launches are recorded and issued as one CUDA graph launch.  The
+ * library keeps an executable graph per launch sequence met (up to 8): the first step with a
+ * new sequence builds and instantiates it, later steps give its kernel nodes the new arguments
+ * (page ids, plan) and relaunch it.  Results are bit-identical to use_graph = 0.  The graphs
+ * live until svt_destroy_cache; calls on one cache must come from one host thread.
+ * Errors: as the calls it makes; the host bookkeeping of the sub-steps that succeeded stands
+ * and their kernels are issued. */
+SVT_API int svt_frame_step(svt_cache* c, int stream, const void* const* k, const void* const* v,
+                           const void* const* q, void* const* out, int use_graph, svt_stream_t s);
+
+/* Graphs built and graph replays (node updates + relaunch) by svt_frame_step so far. */
+SVT_API int svt_get_graph_counts(const svt_cache* c, int* builds, int* replays);
 
 /* Cache statistics of one stream.  [P3] Sec. Implementation Examples. */
 SVT_API int svt_get_cache_stats(const svt_cache* c, int stream, svt_stats* out);

@@ -22,7 +22,8 @@ EXPORTED = [
     "svt_set_free_lists", "svt_append_frame", "svt_evict_frames", "svt_set_defer_eviction",
     "svt_execute_deferred_eviction", "svt_rollback_last_frame", "svt_build_visible_page_table",
     "svt_get_page_table", "svt_read_device_page_table", "svt_plan", "svt_get_plan_info",
-    "svt_run", "svt_get_cache_stats", "svt_device_error", "svt_last_error",
+    "svt_run", "svt_frame_step", "svt_get_graph_counts", "svt_get_cache_stats",
+    "svt_device_error", "svt_last_error",
     "svt_attention_noalloc", "svt_noalloc_device_error", "svt_selftest_wait_limit",
 ]
 
@@ -34,7 +35,7 @@ class CacheOpts(ctypes.Structure):
         ("patch_pages", ctypes.c_int), ("max_qo_len", ctypes.c_int),
         ("max_splits", ctypes.c_int), ("rope_grid", ctypes.c_int),
         ("rope_theta", ctypes.c_float), ("host_only", ctypes.c_int),
-        ("pool", ctypes.c_void_p),
+        ("pool", ctypes.c_void_p), ("no_cross_frame_special", ctypes.c_int),
     ]
 
 
@@ -84,6 +85,8 @@ def load() -> ctypes.CDLL:
         "svt_plan": (I, [VP, i32p, VP]),
         "svt_get_plan_info": (I, [VP, P(PlanInfo)]),
         "svt_run": (I, [VP, I, VP, VP, VP, I, VP]),
+        "svt_frame_step": (I, [VP, I, P(VP), P(VP), P(VP), P(VP), I, VP]),
+        "svt_get_graph_counts": (I, [VP, P(I), P(I)]),
         "svt_get_cache_stats": (I, [VP, I, P(Stats)]),
         "svt_device_error": (I, [VP, VP]),
         "svt_last_error": (ctypes.c_char_p, []),

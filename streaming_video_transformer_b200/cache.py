@@ -53,7 +53,8 @@ class PagedKVCache:
                  scale_frames: int, *, num_blocks: int = 1, num_special: int = 6,
                  num_streams: int = 1, dtype: str = "bf16", patch_pages: int = 0,
                  max_qo_len: int = 0, max_splits: int = 16, rope_grid: int = 0,
-                 rope_theta: float = 100.0, host_only: bool = False, device=None):
+                 rope_theta: float = 100.0, host_only: bool = False,
+                 cross_frame_special: bool = True, device=None):
         self._lib = L.load()
         self._h = ctypes.c_void_p(0)
         self.max_pages, self.page_size, self.H, self.D = max_pages, page_size, H, D
@@ -61,12 +62,16 @@ class PagedKVCache:
         self.num_blocks, self.num_special, self.num_streams = num_blocks, num_special, num_streams
         self.dtype = dtype
         self.host_only = host_only
+        self.cross_frame_special = cross_frame_special
+        # tokens per pool page: a frame's specials share its page without retention
+        self.page_tokens = page_size + (0 if cross_frame_special else num_special)
         opts = L.CacheOpts()
         self._lib.svt_default_opts(ctypes.byref(opts))
         opts.num_blocks, opts.num_special, opts.num_streams = num_blocks, num_special, num_streams
         opts.dtype = _DTYPE_CODES[dtype]
         opts.patch_pages, opts.max_qo_len, opts.max_splits = patch_pages, max_qo_len, max_splits
         opts.rope_grid, opts.rope_theta, opts.host_only = rope_grid, rope_theta, int(host_only)
+        opts.no_cross_frame_special = int(not cross_frame_special)
         self.pool = None
         if not host_only:
             torch = _torch()
@@ -75,7 +80,7 @@ class PagedKVCache:
                 raise SvtError(L.SVT_EINVAL, "bad pool shape")
             tdt = {"bf16": torch.bfloat16, "fp16": torch.float16, "fp32": torch.float32}[dtype]
             self.pool = torch.zeros(
-                (num_blocks, max_pages, 2, page_size, H, D), dtype=tdt,
+                (num_blocks, max_pages, 2, self.page_tokens, H, D), dtype=tdt,
                 device=device if device is not None else "cuda")
             opts.pool = self.pool.data_ptr()
         _check(self._lib.svt_create_cache(max_pages, page_size, H, D, sliding_window,
@@ -184,6 +189,26 @@ class PagedKVCache:
         _check(self._lib.svt_run(self._h, block, _ptr(q), _ptr(out), _ptr(lse), int(force_fp32),
                                  _stream_handle(cuda_stream)))
         return out
+
+    def frame_step(self, ks, vs, qs, outs, stream: int = 0, use_graph: bool = True,
+                   cuda_stream=None):
+        """``svt_frame_step``: append the frame of every block, evict, build, plan
+        and run every block in one call (one CUDA graph launch with
+        ``use_graph``).  ``ks, vs, qs, outs``: one device tensor per block."""
+        L_ = self.num_blocks
+        if not (len(ks) == len(vs) == len(qs) == len(outs) == L_):
+            raise ValueError("one k, v, q and out per block")
+        arr = ctypes.c_void_p * L_
+        ptrs = [arr(*[_ptr(t).value for t in xs]) for xs in (ks, vs, qs, outs)]
+        _check(self._lib.svt_frame_step(self._h, stream, *ptrs, int(use_graph),
+                                        _stream_handle(cuda_stream)))
+        return outs
+
+    def graph_counts(self):
+        """(graphs built, graph replays) of ``frame_step``."""
+        b, r = ctypes.c_int(0), ctypes.c_int(0)
+        _check(self._lib.svt_get_graph_counts(self._h, ctypes.byref(b), ctypes.byref(r)))
+        return b.value, r.value
 
     def device_error(self, cuda_stream=None) -> None:
         _check(self._lib.svt_device_error(self._h, _stream_handle(cuda_stream)))

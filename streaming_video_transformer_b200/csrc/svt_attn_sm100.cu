@@ -514,7 +514,8 @@ __global__ void __launch_bounds__(threads_for(D), 2)
 }
 
 template <int D, bool BF16>
-cudaError_t launch_t(const AttnParams& p, const void* tq, const void* tkv, cudaStream_t s) {
+cudaError_t launch_t(const AttnParams& p, const void* tq, const void* tkv, cudaStream_t s,
+                     Recorder* rec) {
   using C = Cfg<D>;
   auto kern = attn_sm100_kernel<D, BF16>;
   static bool configured = false;
@@ -527,8 +528,7 @@ cudaError_t launch_t(const AttnParams& p, const void* tq, const void* tkv, cudaS
   CUtensorMap mq, mkv;
   memcpy(&mq, tq, sizeof(mq));
   memcpy(&mkv, tkv, sizeof(mkv));
-  kern<<<p.total_items, threads_for(D), C::kSmemBytes, s>>>(mq, mkv, p);
-  return cudaGetLastError();
+  return dispatch(rec, kern, p.total_items, threads_for(D), C::kSmemBytes, s, mq, mkv, p);
 }
 
 
@@ -542,13 +542,13 @@ int attn_items_per_stream(int H, int D, int qtiles, int chunks) {
 int attn_ctas_per_sm(int D) { (void)D; return 2; }   // 256 TMEM columns and < 113 KB smem each
 
 cudaError_t launch_attn_sm100(const AttnParams& p, const void* tmap_q, const void* tmap_kv,
-                              int dtype, cudaStream_t s) {
+                              int dtype, cudaStream_t s, Recorder* rec) {
   if (p.total_items == 0) return cudaSuccess;
   const bool bf16 = dtype == SVT_BF16;
-  if (p.D == 64) return bf16 ? launch_t<64, true>(p, tmap_q, tmap_kv, s)
-                             : launch_t<64, false>(p, tmap_q, tmap_kv, s);
-  if (p.D == 128) return bf16 ? launch_t<128, true>(p, tmap_q, tmap_kv, s)
-                              : launch_t<128, false>(p, tmap_q, tmap_kv, s);
+  if (p.D == 64) return bf16 ? launch_t<64, true>(p, tmap_q, tmap_kv, s, rec)
+                             : launch_t<64, false>(p, tmap_q, tmap_kv, s, rec);
+  if (p.D == 128) return bf16 ? launch_t<128, true>(p, tmap_q, tmap_kv, s, rec)
+                              : launch_t<128, false>(p, tmap_q, tmap_kv, s, rec);
   return cudaErrorInvalidValue;
 }
 

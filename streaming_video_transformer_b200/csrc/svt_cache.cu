@@ -12,7 +12,11 @@
 //    Attention Outperforms SDPA Fallback in Streaming Inference", Sec.
 //    Two-Stream Design.)
 //  * special stream: num_special tokens per frame packed continuously over
-//    pages of the same size, never evicted (same sections).
+//    pages of the same size, never evicted (same sections).  Without
+//    cross-frame special retention (kv_cache_cross_frame_special = False,
+//    "How LingBot-Map Uses KV Caching ...", Sec. Configuration Parameters)
+//    a frame's special tokens follow its patch tokens in the frame's own page
+//    and leave with it; there are no special pages then.
 //  * deferred eviction and rollback of the provisional frame ("How LingBot-Map
 //    Uses KV Caching ...", Sec. Flow-Based Keyframe Selection): rollback puts
 //    the pages back at the FRONT of their free lists so that the allocator
@@ -100,6 +104,8 @@ struct svt_cache {
   // shape and options
   int max_pages = 0, P = 0, H = 0, D = 0, W = 0, S = 0;
   int L = 1, ns = 6, n_streams = 1, dtype = SVT_BF16, elem = 2;
+  bool frame_special = false;  // specials stored in the frame's page (no cross-frame retention)
+  int page_tokens = 0;         // tokens per pool page: P, or P + ns with frame_special
   int patch_pages = 0, max_qo = 0, max_splits = 16, rope_grid = 0;
   float rope_theta = 100.f;
   bool host_only = false;
@@ -143,6 +149,19 @@ struct svt_cache {
   alignas(64) CUtensorMap tmap_q;
   const void* tmap_q_ptr = nullptr;
   int tmap_q_rows = -1;
+
+  // frame steps replayed as CUDA graphs (svt_frame_step): the launches of a
+  // step are recorded into `rec` instead of being issued, then handed to an
+  // executable graph whose kernel nodes are given the new arguments.
+  Recorder* rec = nullptr;
+  struct StepGraph {
+    std::vector<const void*> funcs;       // kernel of each node, in launch order
+    cudaGraph_t graph = nullptr;
+    cudaGraphExec_t exec = nullptr;
+    std::vector<cudaGraphNode_t> nodes;
+  };
+  std::vector<StepGraph> graphs;          // one per launch sequence met so far
+  int graph_builds = 0, graph_replays = 0;
 };
 
 namespace {
@@ -151,7 +170,7 @@ size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
 int page_valid_tokens_last(const svt_cache* c, const StreamState& s) {
   if (!s.special_pages.empty()) return int((s.special_tokens - 1) % c->P) + 1;
-  if (!s.scale.empty() || !s.window.empty()) return c->P;
+  if (!s.scale.empty() || !s.window.empty()) return c->page_tokens;
   return 0;
 }
 
@@ -185,11 +204,11 @@ int encode_kv_map(svt_cache* c) {
   auto enc = tensor_map_encoder();
   if (!enc) return fail(SVT_ECUDA, "cuTensorMapEncodeTiled entry point unavailable");
   const cuuint64_t e = c->elem;
-  cuuint64_t dims[5] = {(cuuint64_t)c->D, (cuuint64_t)c->H, (cuuint64_t)c->P, 2,
+  const cuuint64_t pt = (cuuint64_t)c->page_tokens;
+  cuuint64_t dims[5] = {(cuuint64_t)c->D, (cuuint64_t)c->H, pt, 2,
                         (cuuint64_t)c->L * (cuuint64_t)c->max_pages};
-  cuuint64_t strides[4] = {c->D * e, (cuuint64_t)c->H * c->D * e,
-                           (cuuint64_t)c->P * c->H * c->D * e,
-                           2ull * c->P * c->H * c->D * e};
+  cuuint64_t strides[4] = {c->D * e, (cuuint64_t)c->H * c->D * e, pt * c->H * c->D * e,
+                           2ull * pt * c->H * c->D * e};
   cuuint32_t box[5] = {64, 1, (cuuint32_t)attn_tile_n(c->D), 1, 1};
   cuuint32_t estr[5] = {1, 1, 1, 1, 1};
   CUresult r = enc(&c->tmap_kv,
@@ -253,6 +272,29 @@ double simulate(const std::vector<double>& item_cost, int num_sms) {
   return end;
 }
 
+cudaKernelNodeParams node_params(const LaunchRecord& r, std::vector<void*>& argv) {
+  argv = r.argv();
+  cudaKernelNodeParams kp{};
+  kp.func = const_cast<void*>(r.func);
+  kp.gridDim = r.grid;
+  kp.blockDim = r.block;
+  kp.sharedMemBytes = r.smem;
+  kp.kernelParams = argv.data();
+  kp.extra = nullptr;
+  return kp;
+}
+
+// Issues recorded launches one by one (the path a failed step takes, so that
+// the device state follows the host bookkeeping done before the failure).
+cudaError_t issue_directly(const Recorder& rec, cudaStream_t s) {
+  for (const auto& r : rec.launches) {
+    std::vector<void*> argv = r.argv();
+    cudaError_t e = cudaLaunchKernel(r.func, r.grid, r.block, argv.data(), r.smem, s);
+    if (e != cudaSuccess) return e;
+  }
+  return cudaSuccess;
+}
+
 }  // namespace
 
 namespace svt {
@@ -284,7 +326,9 @@ size_t svt_pool_bytes(int max_pages, int page_size, int H, int D, const svt_cach
   if (opts) o = *opts; else svt_default_opts(&o);
   if (max_pages <= 0 || page_size <= 0 || H <= 0 || D <= 0 || o.num_blocks <= 0) return 0;
   if (o.dtype < SVT_BF16 || o.dtype > SVT_FP32) return 0;
-  return (size_t)o.num_blocks * max_pages * 2 * page_size * H * D * elem_size(o.dtype);
+  const int ns = o.num_special < 0 ? 0 : o.num_special;
+  const size_t page_tokens = (size_t)page_size + (o.no_cross_frame_special ? ns : 0);
+  return (size_t)o.num_blocks * max_pages * 2 * page_tokens * H * D * elem_size(o.dtype);
 }
 
 int svt_create_cache(int max_pages, int page_size, int H, int D, int sliding_window,
@@ -313,7 +357,7 @@ int svt_create_cache(int max_pages, int page_size, int H, int D, int sliding_win
   if (patch_pages < need_patch)
     return fail(SVT_EINVAL, "patch_pages %d < num_streams*(scale_frames+sliding_window+1) = %d",
                 patch_pages, need_patch);
-  if (patch_pages >= max_pages)
+  if (patch_pages > max_pages || (patch_pages == max_pages && !o.no_cross_frame_special))
     return fail(SVT_EINVAL, "max_pages %d leaves no special pages after %d patch pages",
                 max_pages, patch_pages);
   if (o.rope_grid < 0 || (o.rope_grid > 0 && o.rope_grid * o.rope_grid != page_size))
@@ -340,6 +384,8 @@ int svt_create_cache(int max_pages, int page_size, int H, int D, int sliding_win
   c->S = scale_frames;
   c->L = o.num_blocks;
   c->ns = o.num_special;
+  c->frame_special = o.no_cross_frame_special != 0;
+  c->page_tokens = page_size + (c->frame_special ? o.num_special : 0);
   c->n_streams = o.num_streams;
   c->dtype = o.dtype;
   c->elem = elem_size(o.dtype);
@@ -414,6 +460,10 @@ int svt_create_cache(int max_pages, int page_size, int H, int D, int sliding_win
 
 int svt_destroy_cache(svt_cache* c) {
   if (!c) return SVT_OK;
+  for (auto& g : c->graphs) {
+    if (g.exec) cudaGraphExecDestroy(g.exec);
+    if (g.graph) cudaGraphDestroy(g.graph);
+  }
   if (c->dmem) cudaFree(c->dmem);
   delete c;
   return SVT_OK;
@@ -478,12 +528,14 @@ int svt_append_frame(svt_cache* c, int block, int stream, const void* k, const v
     if ((int)s.window.size() > c->W)
       return fail(SVT_ESTATE, "window holds %zu > sliding_window frames: call evict_frames "
                               "after each append", s.window.size());
-    // specials: tokens [n0, n0+ns) of the stream's special sequence
+    // specials: tokens [n0, n0+ns) of the stream's special sequence (in the
+    // frame's own page without cross-frame retention: no special pages)
     const int64_t n0 = s.special_tokens;
+    const bool packed = ns && !c->frame_special;
     const int first_pg = int(n0 / P);
-    const int last_pg = ns ? int((n0 + ns - 1) / P) : first_pg - 1;
-    const int n_new = std::max(0, last_pg + 1 - (int)s.special_pages.size());
-    const int n_touch = ns ? last_pg - first_pg + 1 : 0;
+    const int last_pg = packed ? int((n0 + ns - 1) / P) : first_pg - 1;
+    const int n_new = packed ? std::max(0, last_pg + 1 - (int)s.special_pages.size()) : 0;
+    const int n_touch = packed ? last_pg - first_pg + 1 : 0;
     if (n_touch > kMaxSpecialSpan) return fail(SVT_EINVAL, "special tokens span too many pages");
     if (c->patch_free.empty()) return fail(SVT_ENOPAGES, "patch free list is empty");
     if ((int)c->special_free.size() < n_new) return fail(SVT_ENOPAGES, "special free list is empty");
@@ -514,7 +566,7 @@ int svt_append_frame(svt_cache* c, int block, int stream, const void* k, const v
     s.prov_new_sp = n_new;
     s.blocks_done = 0;
     s.cur_patch = page;
-    s.cur_sp_off0 = ns ? int(n0 % P) : 0;
+    s.cur_sp_off0 = packed ? int(n0 % P) : 0;
     s.cur_n_sp = n_touch;
     for (int i = 0; i < n_touch; ++i) s.cur_sp[i] = s.special_pages[first_pg + i];
     mark_dirty(c);
@@ -531,11 +583,14 @@ int svt_append_frame(svt_cache* c, int block, int stream, const void* k, const v
                 s.blocks_done == c->L ? 0 : s.blocks_done);
   }
   if (!c->host_only) {
-    ap.pool_block = c->pool + (size_t)block * c->max_pages * 2 * P * c->H * c->D * c->elem;
+    ap.pool_block =
+        c->pool + (size_t)block * c->max_pages * 2 * c->page_tokens * c->H * c->D * c->elem;
     ap.k = static_cast<const char*>(k);
     ap.v = static_cast<const char*>(v);
     ap.ns = ns;
     ap.P = P;
+    ap.page_tokens = c->page_tokens;
+    ap.frame_special = c->frame_special ? 1 : 0;
     ap.H = c->H;
     ap.D = c->D;
     ap.elem = c->elem;
@@ -545,7 +600,7 @@ int svt_append_frame(svt_cache* c, int block, int stream, const void* k, const v
     for (int i = 0; i < s.cur_n_sp; ++i) ap.sp_pages[i] = s.cur_sp[i];
     ap.rope_tab = c->rope_grid ? c->d_rope_tab : nullptr;
     ap.rope_grid = c->rope_grid;
-    cudaError_t e = launch_append(ap, c->dtype, reinterpret_cast<cudaStream_t>(cs));
+    cudaError_t e = launch_append(ap, c->dtype, reinterpret_cast<cudaStream_t>(cs), c->rec);
     if (e != cudaSuccess) {
       if (block == 0) {  // undo the allocation so that a failed call changes nothing
         s.has_prov = true;
@@ -569,6 +624,7 @@ int svt_evict_frames(svt_cache* c, int stream) {
     c->patch_free.push_back(s.window.front());
     s.window.pop_front();
     s.ring_head = (s.ring_head + 1) % c->ring_cap;
+    if (c->frame_special) s.special_tokens -= c->ns;   // the frame's specials leave too
     changed = true;
   }
   if (changed) {
@@ -673,7 +729,7 @@ int svt_build_visible_page_table(svt_cache* c, svt_stream_t cs) {
       bp.s[i] = BuildStream{(int)s.scale.size(), s.ring_head, (int)s.window.size(),
                             (int)s.special_pages.size(), page_valid_tokens_last(c, s)};
     }
-    cudaError_t e = launch_build_table(bp, reinterpret_cast<cudaStream_t>(cs));
+    cudaError_t e = launch_build_table(bp, reinterpret_cast<cudaStream_t>(cs), c->rec);
     if (e != cudaSuccess) return cuda_fail(e, "table builder launch");
   }
   c->dirty = false;
@@ -714,8 +770,9 @@ int svt_plan(svt_cache* c, const int32_t* qo_len, svt_stream_t) {
   if (!qo_len) return fail(SVT_EINVAL, "qo_len_per_stream is NULL");
   if (c->dirty) return fail(SVT_ESTATE, "cache changed since build_visible_page_table");
   const int P = c->P;
+  const int PT = c->page_tokens;
   const int TN = attn_tile_n(c->D);
-  const int tpp = (P + TN - 1) / TN;
+  const int tpp = (PT + TN - 1) / TN;
   int rows = 0, page_off = 0;
   AttnParams& a = c->attn;
   SimtParams& m = c->simt;
@@ -746,7 +803,7 @@ int svt_plan(svt_cache* c, const int32_t* qo_len, svt_stream_t) {
     rows += qo_len[i];
     page_off += np;
     info.kv_tiles[i] = sp.tiles;
-    info.kv_tokens[i] = np ? (int64_t)(np - 1) * P + lpl : 0;
+    info.kv_tokens[i] = np ? (int64_t)(np - 1) * PT + lpl : 0;
     info.qo_len[i] = qo_len[i];
   }
   if (rows > c->max_qo) return fail(SVT_EINVAL, "total query rows %d > max_qo_len %d", rows, c->max_qo);
@@ -808,7 +865,7 @@ int svt_plan(svt_cache* c, const int32_t* qo_len, svt_stream_t) {
   a.total_items = items;
   a.H = c->H;
   a.D = c->D;
-  a.P = P;
+  a.P = PT;
   a.max_pages = c->max_pages;
   a.indices = c->d_indices;
   a.scale_log2 = (float)(1.4426950408889634 / std::sqrt((double)c->D));
@@ -835,7 +892,7 @@ int svt_plan(svt_cache* c, const int32_t* qo_len, svt_stream_t) {
   m.total_blocks = blocks;
   m.H = c->H;
   m.D = c->D;
-  m.P = P;
+  m.P = PT;
   m.max_pages = c->max_pages;
   m.indices = c->d_indices;
   m.scale = (float)(1.0 / std::sqrt((double)c->D));
@@ -881,18 +938,18 @@ int svt_run(svt_cache* c, int block, const void* q, void* out, float* lse, int f
     rp.elem = c->elem;
     rp.rope_tab = c->d_rope_tab;
     rp.rope_grid = c->rope_grid;
-    e = launch_rope_q(rp, c->dtype, s);
+    e = launch_rope_q(rp, c->dtype, s, c->rec);
     if (e != cudaSuccess) return cuda_fail(e, "rope_q launch");
     qsrc = c->d_qrope;
   }
-  const size_t block_bytes = (size_t)c->max_pages * 2 * c->P * c->H * c->D * c->elem;
+  const size_t block_bytes = (size_t)c->max_pages * 2 * c->page_tokens * c->H * c->D * c->elem;
   if (force_fp32 || c->dtype == SVT_FP32) {
     SimtParams m = c->simt;
     m.pool_block = c->pool + (size_t)block * block_bytes;
     m.q = qsrc;
     m.out = static_cast<float*>(out);
     m.lse = lse;
-    e = launch_attn_simt(m, c->dtype, s);
+    e = launch_attn_simt(m, c->dtype, s, c->rec);
     if (e != cudaSuccess) return cuda_fail(e, "fp32 attention launch");
     return SVT_OK;
   }
@@ -902,10 +959,10 @@ int svt_run(svt_cache* c, int block, const void* q, void* out, float* lse, int f
   a.block_page_base = (int64_t)block * c->max_pages;
   a.out = out;
   a.lse = lse;
-  e = launch_attn_sm100(a, &c->tmap_q, &c->tmap_kv, c->dtype, s);
+  e = launch_attn_sm100(a, &c->tmap_q, &c->tmap_kv, c->dtype, s, c->rec);
   if (e != cudaSuccess) return cuda_fail(e, "attention launch");
   if (c->any_split) {
-    e = launch_merge(a, c->dtype, s);
+    e = launch_merge(a, c->dtype, s, c->rec);
     if (e != cudaSuccess) return cuda_fail(e, "merge launch");
   }
   return SVT_OK;
@@ -923,6 +980,91 @@ int svt_device_error(svt_cache* c, svt_stream_t cs) {
   if (h)
     return fail(SVT_EDEVICE, "device error 0x%x:%s%s%s", h, (h & kErrPageId) ? " page-id" : "",
                 (h & kErrWaitLimit) ? " wait-limit" : "", (h & kErrShape) ? " shape" : "");
+  return SVT_OK;
+}
+
+int svt_frame_step(svt_cache* c, int stream, const void* const* k, const void* const* v,
+                   const void* const* q, void* const* out, int use_graph, svt_stream_t cs) {
+  if (int r = check_stream(c, stream)) return r;
+  if (c->host_only) return fail(SVT_EINVAL, "host-only cache cannot run kernels");
+  if (!k || !v || !q || !out) return fail(SVT_EINVAL, "k, v, q and out must list one pointer per block");
+  for (int b = 0; b < c->L; ++b)
+    if (!k[b] || !v[b] || !q[b] || !out[b]) return fail(SVT_EINVAL, "null pointer for block %d", b);
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(cs);
+  Recorder rec;
+  c->rec = use_graph ? &rec : nullptr;
+  int r = SVT_OK;
+  for (int b = 0; b < c->L && !r; ++b) r = svt_append_frame(c, b, stream, k[b], v[b], cs);
+  if (!r) r = svt_evict_frames(c, stream);
+  if (!r) r = svt_build_visible_page_table(c, cs);
+  if (!r) {
+    std::vector<int32_t> qo(c->n_streams, 0);
+    qo[stream] = c->ns + c->P;
+    r = svt_plan(c, qo.data(), cs);
+  }
+  for (int b = 0; b < c->L && !r; ++b) r = svt_run(c, b, q[b], out[b], nullptr, 0, cs);
+  c->rec = nullptr;
+  if (!use_graph || rec.launches.empty()) return r;
+  if (r) {
+    const std::string msg = g_err;
+    issue_directly(rec, s);
+    g_err = msg;
+    return r;
+  }
+  std::vector<const void*> funcs;
+  for (const auto& x : rec.launches) funcs.push_back(x.func);
+  svt_cache::StepGraph* g = nullptr;
+  for (auto& x : c->graphs)
+    if (x.funcs == funcs) g = &x;
+  std::vector<void*> argv;
+  if (g) {
+    for (size_t i = 0; i < rec.launches.size(); ++i) {
+      cudaKernelNodeParams kp = node_params(rec.launches[i], argv);
+      cudaError_t e = cudaGraphExecKernelNodeSetParams(g->exec, g->nodes[i], &kp);
+      if (e != cudaSuccess) {
+        cudaGetLastError();
+        issue_directly(rec, s);
+        return cuda_fail(e, "graph node update");
+      }
+    }
+    c->graph_replays += 1;
+  } else {
+    if (c->graphs.size() >= 8) {     // keep a few launch sequences
+      cudaGraphExecDestroy(c->graphs.front().exec);
+      cudaGraphDestroy(c->graphs.front().graph);
+      c->graphs.erase(c->graphs.begin());
+    }
+    svt_cache::StepGraph ng;
+    ng.funcs = funcs;
+    cudaError_t e = cudaGraphCreate(&ng.graph, 0);
+    cudaGraphNode_t prev = nullptr;
+    for (size_t i = 0; e == cudaSuccess && i < rec.launches.size(); ++i) {
+      cudaKernelNodeParams kp = node_params(rec.launches[i], argv);
+      cudaGraphNode_t node = nullptr;
+      e = cudaGraphAddKernelNode(&node, ng.graph, prev ? &prev : nullptr, prev ? 1 : 0, &kp);
+      ng.nodes.push_back(node);
+      prev = node;
+    }
+    if (e == cudaSuccess) e = cudaGraphInstantiate(&ng.exec, ng.graph, 0);
+    if (e != cudaSuccess) {
+      if (ng.graph) cudaGraphDestroy(ng.graph);
+      cudaGetLastError();
+      issue_directly(rec, s);
+      return cuda_fail(e, "graph build");
+    }
+    c->graphs.push_back(std::move(ng));
+    g = &c->graphs.back();
+    c->graph_builds += 1;
+  }
+  cudaError_t e = cudaGraphLaunch(g->exec, s);
+  if (e != cudaSuccess) return cuda_fail(e, "graph launch");
+  return SVT_OK;
+}
+
+int svt_get_graph_counts(const svt_cache* c, int* builds, int* replays) {
+  if (!c || !builds || !replays) return fail(SVT_EINVAL, "null argument");
+  *builds = c->graph_builds;
+  *replays = c->graph_replays;
   return SVT_OK;
 }
 

@@ -4,11 +4,79 @@
 
 #include <cstddef>
 #include <cstdint>
+#include <cstdlib>
+#include <cstring>
+#include <memory>
+#include <tuple>
+#include <utility>
+#include <vector>
 #include <cuda_runtime.h>
 
 #include "../../include/svt.h"
 
 namespace svt {
+
+// ------------------------------------------------------- kernel dispatch
+// Every kernel of the library is launched through dispatch(): with no
+// recorder it is launched at once (cudaLaunchKernel on the given stream);
+// with a recorder the launch (function, shape, copies of the arguments) is
+// appended to it instead, so that a frame step can be replayed as a CUDA
+// graph whose kernel nodes take the recorded arguments.
+struct LaunchRecord {
+  const void* func = nullptr;
+  dim3 grid, block;
+  unsigned smem = 0;
+  std::vector<std::shared_ptr<void>> args;   // one 64-byte aligned copy per argument
+  std::vector<void*> argv() const {
+    std::vector<void*> v;
+    for (const auto& a : args) v.push_back(a.get());
+    return v;
+  }
+};
+
+struct Recorder {
+  std::vector<LaunchRecord> launches;
+};
+
+namespace detail {
+template <typename T>
+std::shared_ptr<void> copy_arg(const T& x) {
+  const size_t n = (sizeof(T) + 63) / 64 * 64;
+  void* mem = std::aligned_alloc(64, n);
+  if (!mem) return nullptr;
+  std::memcpy(mem, &x, sizeof(T));
+  return std::shared_ptr<void>(mem, [](void* q) { std::free(q); });
+}
+template <typename Tup, size_t... I>
+void fill_argv(Tup& t, void** argv, std::index_sequence<I...>) {
+  ((argv[I] = static_cast<void*>(&std::get<I>(t))), ...);
+}
+}  // namespace detail
+
+template <typename... A, typename... B>
+cudaError_t dispatch(Recorder* rec, void (*kern)(A...), dim3 grid, dim3 block, unsigned smem,
+                     cudaStream_t s, B&&... in) {
+  static_assert(sizeof...(A) == sizeof...(B), "argument count");
+  std::tuple<std::decay_t<A>...> args(std::forward<B>(in)...);
+  if (!rec) {
+    void* argv[sizeof...(A)];
+    detail::fill_argv(args, argv, std::index_sequence_for<A...>{});
+    cudaError_t e = cudaLaunchKernel(reinterpret_cast<const void*>(kern), grid, block, argv, smem, s);
+    return e;
+  }
+  LaunchRecord r;
+  r.func = reinterpret_cast<const void*>(kern);
+  r.grid = grid;
+  r.block = block;
+  r.smem = smem;
+  bool ok = true;
+  std::apply([&](const auto&... a) {
+    ((r.args.push_back(detail::copy_arg(a)), ok = ok && r.args.back() != nullptr), ...);
+  }, args);
+  if (!ok) return cudaErrorMemoryAllocation;
+  rec->launches.push_back(std::move(r));
+  return cudaSuccess;
+}
 
 constexpr int kMaxSpecialSpan = 8;   // special pages one frame's specials can touch
 constexpr int kTileM = 128;          // query rows per tensor-core tile
@@ -29,7 +97,9 @@ struct AppendParams {
   char* pool_block;          // pool region of this transformer block
   const char* k;             // [Nq][H][D]
   const char* v;
-  int ns, P, H, D, elem;     // elem = bytes per element
+  int ns, P, H, D, elem;     // elem = bytes per element; P = patch rows of a frame
+  int page_tokens;           // tokens per pool page (P, or P + ns with frame_special)
+  int frame_special;         // 1: special rows go to the patch page after the patches
   int patch_page;
   int sp_off0;               // offset of the frame's first special token in sp_pages[0]
   int n_sp;                  // special pages touched by this frame
@@ -42,7 +112,7 @@ struct AppendParams {
   const float2* rope_tab;    // [grid][D/4] (cos, sin), nullptr = no RoPE
   int rope_grid;
 };
-cudaError_t launch_append(const AppendParams& p, int dtype, cudaStream_t s);
+cudaError_t launch_append(const AppendParams& p, int dtype, cudaStream_t s, Recorder* rec);
 
 // ------------------------------------------------------------- RoPE on Q
 struct RopeQParams {
@@ -52,7 +122,7 @@ struct RopeQParams {
   const float2* rope_tab;
   int rope_grid;
 };
-cudaError_t launch_rope_q(const RopeQParams& p, int dtype, cudaStream_t s);
+cudaError_t launch_rope_q(const RopeQParams& p, int dtype, cudaStream_t s, Recorder* rec);
 
 // -------------------------------------------------------- table builder
 struct BuildStream { int n_scale, ring_head, ring_len, n_special, lpl; };
@@ -67,7 +137,7 @@ struct BuildParams {
   unsigned* err;
   BuildStream s[SVT_MAX_STREAMS];
 };
-cudaError_t launch_build_table(const BuildParams& p, cudaStream_t s);
+cudaError_t launch_build_table(const BuildParams& p, cudaStream_t s, Recorder* rec);
 
 // ------------------------------------------------------------ attention
 // Per-stream slice of one attention launch.
@@ -85,7 +155,7 @@ struct StreamPlan {
 
 struct AttnParams {
   int n_streams, total_items;
-  int H, D, P, max_pages;
+  int H, D, P, max_pages;    // P = tokens per pool page
   int64_t block_page_base;   // block * max_pages (page coordinate of this block's page 0)
   const int* indices;        // device visible table
   float scale_log2;          // log2(e) / sqrt(D)
@@ -103,16 +173,16 @@ struct AttnParams {
 int attn_items_per_stream(int H, int D, int qtiles, int chunks);
 int attn_ctas_per_sm(int D);   // resident CTAs of the tensor-core kernel per SM
 cudaError_t launch_attn_sm100(const AttnParams& p, const void* tmap_q, const void* tmap_kv,
-                              int dtype, cudaStream_t s);
+                              int dtype, cudaStream_t s, Recorder* rec);
 
 // Combines split-KV partials into out / lse.
-cudaError_t launch_merge(const AttnParams& p, int dtype, cudaStream_t s);
+cudaError_t launch_merge(const AttnParams& p, int dtype, cudaStream_t s, Recorder* rec);
 
 // fp32-FMA kernel (force_fp32 / fp32 pool).  Writes fp32 out and lse directly.
 struct SimtStream { int q_off, nq, rblocks, page_off, n_pages, lpl, block_off; };
 struct SimtParams {
   int n_streams, total_blocks;
-  int H, D, P, max_pages;
+  int H, D, P, max_pages;    // P = tokens per pool page
   const char* pool_block;
   const int* indices;
   const char* q;
@@ -123,7 +193,7 @@ struct SimtParams {
   SimtStream s[SVT_MAX_STREAMS];
 };
 int simt_rows_per_block(int D);
-cudaError_t launch_attn_simt(const SimtParams& p, int dtype, cudaStream_t s);
+cudaError_t launch_attn_simt(const SimtParams& p, int dtype, cudaStream_t s, Recorder* rec);
 
 // Sets the thread-local message returned by svt_last_error(); returns `code`.
 int report_error(int code, const char* msg);

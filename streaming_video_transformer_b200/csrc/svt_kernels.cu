@@ -51,18 +51,24 @@ __device__ __forceinline__ void rope_pair(uint4& lo, uint4& hi, const float2* ta
   }
 }
 
-// One 16-byte vector `vi` of row `row` of a frame: where it lands in the pool.
+// Row `row` of a frame: where it lands in the pool.  Patch rows go to
+// offsets 0..P-1 of the frame's page; special rows either continue the
+// stream's packed special pages or, without cross-frame retention, follow the
+// patches in the frame's own page.
 __device__ __forceinline__ size_t pool_offset(const AppendParams& p, int kv, int row, size_t row_bytes) {
   int page, off;
-  if (row < p.ns) {
+  if (row < p.ns && !p.frame_special) {
     const int n = p.sp_off0 + row;
     page = p.sp_pages[n / p.P];
     off = n % p.P;
+  } else if (row < p.ns) {
+    page = p.patch_page;
+    off = p.P + row;
   } else {
     page = p.patch_page;
     off = row - p.ns;
   }
-  return ((size_t)(page * 2 + kv) * p.P + off) * row_bytes;
+  return ((size_t)(page * 2 + kv) * p.page_tokens + off) * row_bytes;
 }
 
 template <typename T>
@@ -330,15 +336,14 @@ __global__ void __launch_bounds__(kSimtThreads) attn_simt_kernel(SimtParams p) {
 }
 
 template <typename T>
-cudaError_t launch_simt_t(const SimtParams& p, cudaStream_t s) {
+cudaError_t launch_simt_t(const SimtParams& p, cudaStream_t s, Recorder* rec) {
   if (p.total_blocks == 0) return cudaSuccess;
   switch (p.D) {
-    case 32: attn_simt_kernel<T, 32><<<p.total_blocks, kSimtThreads, 0, s>>>(p); break;
-    case 64: attn_simt_kernel<T, 64><<<p.total_blocks, kSimtThreads, 0, s>>>(p); break;
-    case 128: attn_simt_kernel<T, 128><<<p.total_blocks, kSimtThreads, 0, s>>>(p); break;
+    case 32: return dispatch(rec, attn_simt_kernel<T, 32>, p.total_blocks, kSimtThreads, 0, s, p);
+    case 64: return dispatch(rec, attn_simt_kernel<T, 64>, p.total_blocks, kSimtThreads, 0, s, p);
+    case 128: return dispatch(rec, attn_simt_kernel<T, 128>, p.total_blocks, kSimtThreads, 0, s, p);
     default: return cudaErrorInvalidValue;
   }
-  return cudaGetLastError();
 }
 
 int grid_for(long work, int threads) {
@@ -350,34 +355,31 @@ int grid_for(long work, int threads) {
 
 int simt_rows_per_block(int D) { return kSimtThreads / (D / 32); }
 
-cudaError_t launch_append(const AppendParams& p, int dtype, cudaStream_t s) {
+cudaError_t launch_append(const AppendParams& p, int dtype, cudaStream_t s, Recorder* rec) {
   const long vecs = (long)(p.ns + p.P) * p.H * p.D * p.elem / 16;
   dim3 grid(grid_for(vecs, 256), 2);
   switch (dtype) {
-    case SVT_BF16: append_kernel<__nv_bfloat16><<<grid, 256, 0, s>>>(p); break;
-    case SVT_FP16: append_kernel<__half><<<grid, 256, 0, s>>>(p); break;
-    default: append_kernel<float><<<grid, 256, 0, s>>>(p); break;
+    case SVT_BF16: return dispatch(rec, append_kernel<__nv_bfloat16>, grid, 256, 0, s, p);
+    case SVT_FP16: return dispatch(rec, append_kernel<__half>, grid, 256, 0, s, p);
+    default: return dispatch(rec, append_kernel<float>, grid, 256, 0, s, p);
   }
-  return cudaGetLastError();
 }
 
-cudaError_t launch_rope_q(const RopeQParams& p, int dtype, cudaStream_t s) {
+cudaError_t launch_rope_q(const RopeQParams& p, int dtype, cudaStream_t s, Recorder* rec) {
   const long vecs = (long)p.rows * p.H * p.D * p.elem / 16;
   const int grid = grid_for(vecs, 256);
   switch (dtype) {
-    case SVT_BF16: rope_q_kernel<__nv_bfloat16><<<grid, 256, 0, s>>>(p); break;
-    case SVT_FP16: rope_q_kernel<__half><<<grid, 256, 0, s>>>(p); break;
-    default: rope_q_kernel<float><<<grid, 256, 0, s>>>(p); break;
+    case SVT_BF16: return dispatch(rec, rope_q_kernel<__nv_bfloat16>, grid, 256, 0, s, p);
+    case SVT_FP16: return dispatch(rec, rope_q_kernel<__half>, grid, 256, 0, s, p);
+    default: return dispatch(rec, rope_q_kernel<float>, grid, 256, 0, s, p);
   }
-  return cudaGetLastError();
 }
 
-cudaError_t launch_build_table(const BuildParams& p, cudaStream_t s) {
-  build_table_kernel<<<1, 256, 0, s>>>(p);
-  return cudaGetLastError();
+cudaError_t launch_build_table(const BuildParams& p, cudaStream_t s, Recorder* rec) {
+  return dispatch(rec, build_table_kernel, 1, 256, 0, s, p);
 }
 
-cudaError_t launch_merge(const AttnParams& p, int dtype, cudaStream_t s) {
+cudaError_t launch_merge(const AttnParams& p, int dtype, cudaStream_t s, Recorder* rec) {
   int rows = 0;
   for (int i = 0; i < p.n_streams; ++i) rows += p.s[i].nq;
   const int tpp = p.D / 4;
@@ -385,18 +387,15 @@ cudaError_t launch_merge(const AttnParams& p, int dtype, cudaStream_t s) {
   const long pairs = (long)rows * p.H;
   const int grid = (int)((pairs + pairs_per_block - 1) / pairs_per_block);
   if (grid == 0) return cudaSuccess;
-  if (dtype == SVT_BF16)
-    merge_kernel<__nv_bfloat16><<<grid, 128, 0, s>>>(p);
-  else
-    merge_kernel<__half><<<grid, 128, 0, s>>>(p);
-  return cudaGetLastError();
+  if (dtype == SVT_BF16) return dispatch(rec, merge_kernel<__nv_bfloat16>, grid, 128, 0, s, p);
+  return dispatch(rec, merge_kernel<__half>, grid, 128, 0, s, p);
 }
 
-cudaError_t launch_attn_simt(const SimtParams& p, int dtype, cudaStream_t s) {
+cudaError_t launch_attn_simt(const SimtParams& p, int dtype, cudaStream_t s, Recorder* rec) {
   switch (dtype) {
-    case SVT_BF16: return launch_simt_t<__nv_bfloat16>(p, s);
-    case SVT_FP16: return launch_simt_t<__half>(p, s);
-    default: return launch_simt_t<float>(p, s);
+    case SVT_BF16: return launch_simt_t<__nv_bfloat16>(p, s, rec);
+    case SVT_FP16: return launch_simt_t<__half>(p, s, rec);
+    default: return launch_simt_t<float>(p, s, rec);
   }
 }
 

@@ -6,6 +6,11 @@ and special pages patch_pages..max_pages-1 sit in two FIFO free lists handed
 out from the front; evicted window pages go to the back; a rolled-back frame
 returns its pages to the front.  This model restates that policy in plain
 Python so that the library's tables can be checked bit for bit.
+
+Without cross-frame special retention each frame's special tokens sit after
+its patch tokens in the frame's own page (page_size + num_special tokens), so
+no special pages are used, eviction drops a frame's specials with its patches,
+and every visible page is full.
 """
 from collections import deque
 
@@ -20,8 +25,10 @@ class StreamModel:
 
 
 class AllocModel:
-    def __init__(self, max_pages, P, ns, S, W, num_streams=1, patch_pages=0):
+    def __init__(self, max_pages, P, ns, S, W, num_streams=1, patch_pages=0,
+                 cross_frame_special=True):
         self.max_pages, self.P, self.ns, self.S, self.W = max_pages, P, ns, S, W
+        self.cross = cross_frame_special
         self.patch_pages = patch_pages or num_streams * (S + W + 1)
         self.patch_free = deque(range(self.patch_pages))
         self.special_free = deque(range(self.patch_pages, max_pages))
@@ -32,7 +39,7 @@ class AllocModel:
         assert st.prov is None and len(st.window) <= self.W
         n0 = st.special_tokens
         last_pg = (n0 + self.ns - 1) // self.P if self.ns else -1
-        n_new = max(0, last_pg + 1 - len(st.special))
+        n_new = max(0, last_pg + 1 - len(st.special)) if self.cross else 0
         if not self.patch_free or len(self.special_free) < n_new:
             raise MemoryError
         page = self.patch_free.popleft()
@@ -51,6 +58,8 @@ class AllocModel:
             return
         while len(st.window) > self.W:
             self.patch_free.append(st.window.popleft())
+            if not self.cross:
+                st.special_tokens -= self.ns
 
     def accept(self, s):
         st = self.st[s]
@@ -77,7 +86,7 @@ class AllocModel:
             if st.special:
                 lpl.append((st.special_tokens - 1) % self.P + 1)
             elif st.scale or st.window:
-                lpl.append(self.P)
+                lpl.append(self.P if self.cross else self.P + self.ns)
             else:
                 lpl.append(0)
         return indptr, indices, lpl

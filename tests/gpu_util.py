@@ -47,6 +47,11 @@ def make_cache(w, max_pages, num_streams=1, **kw):
                         rope_grid=w.rope_grid, rope_theta=w.rope_theta, **kw)
 
 
+def oracle_stream_for(cache, w):
+    """The oracle stream matching a cache's special-token retention."""
+    return FrameStream(w.P, w.ns, w.S, w.W, cross_frame_special=cache.cross_frame_special)
+
+
 class FrameBank:
     """The R distinct data frames of (block, stream), on the device and as
     float64 oracle inputs (with RoPE applied to the patch rows of Q and K
@@ -91,7 +96,7 @@ def gather_visible(cache, block, stream, dev_table=True):
     pool = cache.pool[block]                                  # [max_pages, 2, P, H, D]
     sel = pool[torch.as_tensor(pages, dtype=torch.long, device=pool.device)]
     n = len(pages)
-    k = sel[:, 0].reshape(n * cache.page_size, cache.H, cache.D)
-    v = sel[:, 1].reshape(n * cache.page_size, cache.H, cache.D)
-    ntok = (n - 1) * cache.page_size + int(lp[stream])
+    k = sel[:, 0].reshape(n * cache.page_tokens, cache.H, cache.D)
+    v = sel[:, 1].reshape(n * cache.page_tokens, cache.H, cache.D)
+    ntok = (n - 1) * cache.page_tokens + int(lp[stream])
     return k[:ntok].double().cpu().numpy(), v[:ntok].double().cpu().numpy()

@@ -1,0 +1,167 @@
+"""GPU parity without cross-frame special retention
+(kv_cache_cross_frame_special = False): a frame's special tokens are visible
+exactly while its patch tokens are, and are stored after them in the frame's
+own page.  Tables, pool bytes and outputs against the allocator model and the
+oracle, from the tiny stream up to the ViT-L-sized step."""
+import numpy as np
+import pytest
+import torch
+
+import golden_io
+from alloc_model import AllocModel
+from gpu_util import (FrameBank, assert_close, gather_visible, make_cache, oracle_out,
+                      oracle_stream_for)
+from streaming_video_transformer_b200.inputs import WORKLOADS, small_workload
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _build():
+    from streaming_video_transformer_b200.build import build
+    build()
+
+
+def _pages(w, streams=1):
+    return streams * (w.S + w.W + 1)
+
+
+def _frame(c, w, bank, t, stream=0, deferred=False):
+    q, k, v = bank.device(t)
+    c.set_defer_eviction(deferred, stream)
+    for b in range(w.blocks):
+        c.append_frame(b, k, v, stream=stream)
+    c.evict_frames(stream)
+    return q
+
+
+def _check_step(c, w, st, m, q, q64, what):
+    c.build_visible_page_table()
+    c.plan([w.Nq])
+    dip, dix, dlp = c.read_device_page_table()
+    hip, hix, hlp = c.get_page_table()
+    mip, mix, mlp = m.table()
+    assert list(dip) == list(hip) == mip and list(dix) == list(hix) == mix, what
+    assert list(dlp) == list(hlp) == mlp, what
+    gk, gv = gather_visible(c, 0, 0)
+    ok, ov = st.visible_kv()
+    assert gk.shape[0] == st.num_visible_tokens()
+    assert np.array_equal(gk, ok) and np.array_equal(gv, ov), what
+    ref, ref_lse = oracle_out(st, q64)
+    lse = torch.empty((w.Nq, w.H), dtype=torch.float32, device="cuda")
+    assert_close(c.run(0, q, lse=lse), ref, what=what)
+    np.testing.assert_allclose(lse.cpu().numpy(), ref_lse, atol=2e-2)
+    assert_close(c.run(0, q, force_fp32=True), ref, fp32=True, what="fp32 " + what)
+
+
+CASES = [
+    dict(P=16, ns=6, S=2, W=4, H=2, D=64, frames=12),                       # the tiny stream
+    dict(P=122, ns=6, S=1, W=3, H=2, D=64, frames=7),                       # 128-token pages
+    dict(P=250, ns=6, S=2, W=2, H=3, D=64, frames=6),                       # 2 tiles + tail
+    dict(P=64, ns=6, S=0, W=3, H=2, D=128, frames=6, dtype="fp16"),         # no scale frames
+    dict(P=100, ns=6, S=1, W=0, H=2, D=128, frames=4, rope_grid=10),        # empty window, RoPE
+    dict(P=36, ns=6, S=2, W=2, H=2, D=64, frames=6, rope_grid=6, dtype="fp32"),
+]
+
+
+@pytest.mark.parametrize("cfg", CASES, ids=[str(i) for i in range(len(CASES))])
+def test_stream_every_frame(cfg):
+    w = small_workload(**cfg, R=cfg["frames"])
+    c = make_cache(w, _pages(w), cross_frame_special=False)
+    m = AllocModel(_pages(w), w.P, w.ns, w.S, w.W, cross_frame_special=False)
+    bank = FrameBank(w, 0, 0)
+    st = oracle_stream_for(c, w)
+    for t in range(w.frames):
+        q = _frame(c, w, bank, t)
+        m.append(0); m.evict(0)
+        q64, k64, v64 = bank.oracle(t)
+        st.append_frame(k64, v64)
+        _check_step(c, w, st, m, q, q64, f"{cfg} t={t + 1}")
+        s = c.get_cache_stats()
+        assert s["special_tokens"] == w.ns * (s["scale_pages"] + s["live_pages"])
+    c.device_error()
+
+
+def test_hand_worked_example_without_retention():
+    """The two-frame closed form without retention, embedded in D=64 as in the
+    retained case (q scaled by 4 so that q.k/sqrt(64) = the example's q.k/2)."""
+    cases, _ = golden_io.two_frame_cases(cross_frame_special=False)
+    D = 64
+
+    def pad(rows):
+        x = torch.zeros((3, 1, D), dtype=torch.bfloat16)
+        for i, r in enumerate(rows):
+            x[i, 0, :4] = torch.tensor(r, dtype=torch.bfloat16)
+        return x.cuda()
+
+    q = pad([[8, 0, 0, 0], [0] * 4, [0] * 4])
+    f0 = (pad([[1, 0, 0, 0], [0] * 4, [0] * 4]), pad([[1, 0, 0, 0], [0, 1, 0, 0], [0, 0, 1, 0]]))
+    f1 = (pad([[0] * 4, [1, 0, 0, 0], [0] * 4]), pad([[0, 0, 0, 1], [1, 1, 0, 0], [0] * 4]))
+    for S, W, t, row, expected in cases:
+        w = small_workload(P=2, ns=1, S=S, W=W, H=1, D=D)
+        c = make_cache(w, max_pages=S + W + 1, cross_frame_special=False)
+        for k, v in (f0, f1)[:t]:
+            c.append_frame(0, k, v)
+            c.evict_frames()
+        c.build_visible_page_table()
+        c.plan([3])
+        out = c.run(0, q).float().cpu().numpy()
+        np.testing.assert_allclose(out[row, 0, :4], expected, atol=4e-3)
+        out32 = c.run(0, q, force_fp32=True).cpu().numpy()
+        np.testing.assert_allclose(out32[row, 0, :4], expected, atol=1e-6)
+
+
+def test_deferred_frames_and_rollback():
+    """Every third frame deferred, half of them rejected: the provisional
+    frame's specials are visible with it and leave with a rollback; accepted
+    frames evict the oldest window frame with its specials."""
+    w = small_workload(P=40, ns=6, S=2, W=3, H=2, D=64, R=16, frames=16)
+    c = make_cache(w, _pages(w), cross_frame_special=False)
+    m = AllocModel(_pages(w), w.P, w.ns, w.S, w.W, cross_frame_special=False)
+    bank = FrameBank(w, 0, 0)
+    st = oracle_stream_for(c, w)
+    rng = np.random.default_rng(42)
+    for t in range(w.frames):
+        deferred = t % 3 == 2
+        m.st[0].defer = deferred
+        q = _frame(c, w, bank, t, deferred=deferred)
+        m.append(0); m.evict(0)
+        q64, k64, v64 = bank.oracle(t)
+        st.append_frame(k64, v64, deferred=deferred)
+        _check_step(c, w, st, m, q, q64, f"t={t + 1} deferred={deferred}")
+        if deferred:
+            if rng.random() < 0.5:
+                c.rollback_last_frame(); m.rollback(0); st.rollback_last_frame()
+            else:
+                c.execute_deferred_eviction(); m.accept(0); st.execute_deferred_eviction()
+    c.device_error()
+
+
+def test_vitl_step_full_size_without_retention():
+    """ViT-L-sized step (H16, D64, 1369 patches, S8, W64) at t = 120 frames:
+    72 visible frames of 1375 tokens each (99,000 keys), sampled rows against
+    the oracle, the pool bit for bit, and the table against the model."""
+    w = WORKLOADS["vitl_step"]
+    frames = 120
+    c = make_cache(w, _pages(w), cross_frame_special=False)
+    m = AllocModel(_pages(w), w.P, w.ns, w.S, w.W, cross_frame_special=False)
+    bank = FrameBank(w, 0, 0)
+    st = oracle_stream_for(c, w)
+    for t in range(frames):
+        q = _frame(c, w, bank, t)
+        m.append(0); m.evict(0)
+        st.append_frame(*bank.oracle(t)[1:])
+    c.build_visible_page_table()
+    c.plan([w.Nq])
+    assert list(c.get_page_table()[1]) == m.table()[1]
+    info = c.plan_info()
+    assert info["kv_tokens"][0] == st.num_visible_tokens() == 72 * 1375
+    assert info["kv_tiles"][0] == 72 * 11
+    rows = np.array(sorted({0, 3, 5, 6, 127, 128, 640, 1279, 1280, 1374}))
+    ref, _ = oracle_out(st, bank.oracle(frames - 1)[0], rows)
+    assert_close(c.run(0, q)[rows], ref, what="bf16")
+    assert_close(c.run(0, q, force_fp32=True)[rows], ref, fp32=True, what="fp32")
+    gk, gv = gather_visible(c, 0, 0)
+    ok, ov = st.visible_kv()
+    assert np.array_equal(gk, ok) and np.array_equal(gv, ov)
+    c.device_error()

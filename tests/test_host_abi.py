@@ -55,16 +55,17 @@ def _check_against(c, m):
         assert c.get_cache_stats(s) == m.stats(s)
 
 
+@pytest.mark.parametrize("cross", [True, False])
 @pytest.mark.parametrize("seed", range(6))
-def test_random_op_sequences_match_model(seed):
+def test_random_op_sequences_match_model(seed, cross):
     rng = np.random.default_rng(seed)
     ns_ = int(rng.integers(1, 4))
     P, ns, S, W = int(rng.integers(3, 7)), int(rng.integers(0, 4)), int(rng.integers(0, 3)), int(rng.integers(0, 4))
     ns = min(ns, P)
-    max_pages = ns_ * (S + W + 1) + 30
+    max_pages = ns_ * (S + W + 1) + (30 if cross else 0)
     c = _host_cache(max_pages=max_pages, page_size=P, num_special=ns, scale_frames=S,
-                    sliding_window=W, num_streams=ns_, num_blocks=2)
-    m = AllocModel(max_pages, P, ns, S, W, ns_)
+                    sliding_window=W, num_streams=ns_, num_blocks=2, cross_frame_special=cross)
+    m = AllocModel(max_pages, P, ns, S, W, ns_, cross_frame_special=cross)
     for step in range(120):
         s = int(rng.integers(0, ns_))
         st = m.st[s]
@@ -114,6 +115,49 @@ def test_two_frame_example_page_table():
     npatch = c.patch_pages
     assert list(ix) == [npatch if x == "NPATCH" else int(x) for x in idx]
     assert list(lp) == [lpl]
+
+
+def test_two_frame_example_page_table_without_cross_frame_special():
+    _, tables = golden_io.two_frame_cases(cross_frame_special=False)
+    (S, W, t, idx, lpl), = tables
+    c = _host_cache(max_pages=12, page_size=2, num_special=1, scale_frames=S, sliding_window=W,
+                    cross_frame_special=False)
+    for _ in range(t):
+        c.append_frame(0)
+        c.evict_frames()
+    ip, ix, lp = c.get_page_table()
+    assert list(ix) == [int(x) for x in idx]
+    assert list(lp) == [lpl]
+
+
+def test_no_cross_frame_special_counts_and_pool_size():
+    """Without retention: the tiny stream's visible counts (golden), the
+    special-token statistic (the specials of resident frames only), a pool
+    with no special pages at all, and pool pages of page_size + num_special
+    tokens."""
+    vc = golden_io.visible_counts()
+    counts = [int(x) for x in vc["tiny_nocross"][1]]
+    P, ns, S, W = 16, 6, 2, 4
+    c = _host_cache(max_pages=S + W + 1, page_size=P, num_special=ns, scale_frames=S,
+                    sliding_window=W, cross_frame_special=False)
+    for t in range(1, 13):
+        c.append_frame(0)
+        c.evict_frames()
+        ip, ix, lp = c.get_page_table()
+        assert (len(ix) - 1) * (P + ns) + lp[0] == counts[t - 1]
+        st = c.get_cache_stats()
+        assert st["special_tokens"] == ns * (st["scale_pages"] + st["live_pages"])
+    with pytest.raises(SvtError):                            # cross retention needs special pages
+        _host_cache(max_pages=S + W + 1, page_size=P, num_special=ns, scale_frames=S,
+                    sliding_window=W)
+    lib = _lib.load()
+    opts = _lib.CacheOpts()
+    lib.svt_default_opts(ctypes.byref(opts))
+    assert opts.no_cross_frame_special == 0
+    opts.num_special = ns
+    base = lib.svt_pool_bytes(10, P, 2, 64, ctypes.byref(opts))
+    opts.no_cross_frame_special = 1
+    assert lib.svt_pool_bytes(10, P, 2, 64, ctypes.byref(opts)) == base * (P + ns) // P
 
 
 def test_steady_state_page_counts():
