@@ -358,7 +358,7 @@ def run_secondary(args):
         fr = [[x.to(dev) for x in frame_qkv(w, 0, 0, t)] for t in range(w.frames)]
         out = torch.empty_like(fr[0][0])
 
-        def stream_once():
+        def separate_calls():
             c.reset()
             for t in range(w.frames):
                 q, k, v = fr[t]
@@ -367,19 +367,37 @@ def run_secondary(args):
                 c.build_visible_page_table()
                 c.plan([w.Nq])
                 c.run(0, q, out=out)
-        for _ in range(args.warmup):
-            stream_once()
-        torch.cuda.synchronize()
-        a, b = ev(), ev()
-        a.record()
-        for _ in range(args.steps):
-            stream_once()
-        b.record()
-        torch.cuda.synchronize()
-        ms = a.elapsed_time(b)
+
+        def one_call(use_graph):
+            def f():
+                c.reset()
+                for t in range(w.frames):
+                    q, k, v = fr[t]
+                    c.frame_step([k], [v], [q], [out], use_graph=use_graph)
+            return f
+
+        variants = {"separate_calls": separate_calls, "frame_step": one_call(False),
+                    "frame_step_graph": one_call(True)}
+        us = {}
+        for name, fn in variants.items():
+            for _ in range(args.warmup):
+                fn()
+            torch.cuda.synchronize()
+            a, b = ev(), ev()
+            a.record()
+            for _ in range(args.steps):
+                fn()
+            b.record()
+            torch.cuda.synchronize()
+            us[name] = 1e3 * a.elapsed_time(b) / (args.steps * w.frames)
+        builds, replays = c.graph_counts()
         line.update(metric="frames/s (12-frame stream, full frame step)",
-                    value=args.steps * w.frames / (ms / 1e3), unit="frames/s",
-                    us_per_frame=1e3 * ms / (args.steps * w.frames), steps=args.steps)
+                    value=1e6 / us["frame_step_graph"], unit="frames/s",
+                    us_per_frame=us, steps=args.steps,
+                    note="value: svt_frame_step with CUDA-graph replay (one call and one graph "
+                         "launch per frame); us_per_frame also gives the five separate calls "
+                         "and svt_frame_step without a graph",
+                    graphs={"built": builds, "replays": replays})
     elif args.workload == "ragged4":
         ages = list(w.ages)
         c = make(w, ages, streams=4)
