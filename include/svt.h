@@ -215,6 +215,17 @@ SVT_API int svt_read_device_page_table(svt_cache* c, int32_t* indptr, int32_t* i
  * visible tokens), SVT_EINVAL (total rows > max_qo_len). */
 SVT_API int svt_plan(svt_cache* c, const int32_t* qo_len_per_stream, svt_stream_t s);
 
+/* As svt_plan, with a dense K/V segment per stream attended after its visible pages:
+ * extra_len[num_streams] host array of segment rows (NULL or 0 = none; with RoPE whole frames).
+ * This is the skip-append step for non-keyframes ([P1] Sec. Implementation Examples; [P3]
+ * Sec. Flow-Based Keyframe Selection): the frame's queries attend to the cache plus the frame's
+ * own K/V, which is never written to the pool -- the allocator, the page table and the pool
+ * stay untouched.  Run the plan with svt_run_extra.  Segment rows of all streams are
+ * concatenated in stream order, at most max_qo_len in total.
+ * Errors: as svt_plan; SVT_EINVAL for a segment on a stream without queries. */
+SVT_API int svt_plan_extra(svt_cache* c, const int32_t* qo_len_per_stream, const int32_t* extra_len,
+                           svt_stream_t s);
+
 /* Plan summary (work items, splits, tiles) for tests and benchmarks. */
 SVT_API int svt_get_plan_info(const svt_cache* c, svt_plan_info* out);
 
@@ -233,6 +244,15 @@ SVT_API int svt_get_plan_info(const svt_cache* c, svt_plan_info* out);
  * planned stream), SVT_EINVAL, SVT_ECUDA. */
 SVT_API int svt_run(svt_cache* c, int block, const void* q, void* out, float* lse, int force_fp32,
             svt_stream_t s);
+
+/* svt_run for a plan made by svt_plan_extra: k_extra, v_extra are DEVICE [sum extra_len][H][D]
+ * arrays in the cache dtype (16-byte aligned), the K and V rows of every stream's segment,
+ * concatenated in stream order.  With RoPE the segment's K patch rows are rotated like
+ * appended keys (into library scratch; the caller's array is not modified).  A stream with a
+ * segment needs no append of the current frame in `block`.  k_extra and v_extra must be NULL
+ * exactly when the plan has no segment.  Errors: as svt_run. */
+SVT_API int svt_run_extra(svt_cache* c, int block, const void* q, const void* k_extra,
+                          const void* v_extra, void* out, float* lse, int force_fp32, svt_stream_t s);
 
 /* One whole frame step of one stream, from a single call: for every block b the frame's
  * k[b], v[b] are appended (svt_append_frame), then svt_evict_frames, svt_build_visible_page_table

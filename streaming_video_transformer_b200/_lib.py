@@ -21,8 +21,8 @@ EXPORTED = [
     "svt_default_opts", "svt_pool_bytes", "svt_create_cache", "svt_destroy_cache", "svt_reset",
     "svt_set_free_lists", "svt_append_frame", "svt_evict_frames", "svt_set_defer_eviction",
     "svt_execute_deferred_eviction", "svt_rollback_last_frame", "svt_build_visible_page_table",
-    "svt_get_page_table", "svt_read_device_page_table", "svt_plan", "svt_get_plan_info",
-    "svt_run", "svt_frame_step", "svt_get_graph_counts", "svt_get_cache_stats",
+    "svt_get_page_table", "svt_read_device_page_table", "svt_plan", "svt_plan_extra",
+    "svt_get_plan_info", "svt_run", "svt_run_extra", "svt_frame_step", "svt_get_graph_counts", "svt_get_cache_stats",
     "svt_device_error", "svt_last_error",
     "svt_attention_noalloc", "svt_noalloc_device_error", "svt_selftest_wait_limit",
 ]
@@ -83,8 +83,10 @@ def load() -> ctypes.CDLL:
         "svt_get_page_table": (I, [VP, i32p, i32p, i32p, I, P(I)]),
         "svt_read_device_page_table": (I, [VP, i32p, i32p, i32p, I, P(I), VP]),
         "svt_plan": (I, [VP, i32p, VP]),
+        "svt_plan_extra": (I, [VP, i32p, i32p, VP]),
         "svt_get_plan_info": (I, [VP, P(PlanInfo)]),
         "svt_run": (I, [VP, I, VP, VP, VP, I, VP]),
+        "svt_run_extra": (I, [VP, I, VP, VP, VP, VP, VP, I, VP]),
         "svt_frame_step": (I, [VP, I, P(VP), P(VP), P(VP), P(VP), I, VP]),
         "svt_get_graph_counts": (I, [VP, P(I), P(I)]),
         "svt_get_cache_stats": (I, [VP, I, P(Stats)]),

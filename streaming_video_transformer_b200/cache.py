@@ -165,12 +165,22 @@ class PagedKVCache:
         return ip, ix[:n.value].copy(), lp
 
     # ------------------------------------------------------- plan / run
-    def plan(self, qo_len_per_stream, cuda_stream=None) -> None:
+    def plan(self, qo_len_per_stream, extra_len=None, cuda_stream=None) -> None:
+        """``svt_plan``, or ``svt_plan_extra`` when ``extra_len`` (rows of a dense
+        K/V segment per stream, attended without being stored) is given."""
         q = np.ascontiguousarray(qo_len_per_stream, dtype=np.int32)
         if len(q) != self.num_streams:
             raise ValueError("one qo_len per stream")
         cs = ctypes.c_void_p(0) if self.host_only else _stream_handle(cuda_stream)
-        _check(self._lib.svt_plan(self._h, q.ctypes.data_as(ctypes.POINTER(ctypes.c_int32)), cs))
+        p32 = ctypes.POINTER(ctypes.c_int32)
+        if extra_len is None:
+            _check(self._lib.svt_plan(self._h, q.ctypes.data_as(p32), cs))
+        else:
+            x = np.ascontiguousarray(extra_len, dtype=np.int32)
+            if len(x) != self.num_streams:
+                raise ValueError("one extra_len per stream")
+            _check(self._lib.svt_plan_extra(self._h, q.ctypes.data_as(p32), x.ctypes.data_as(p32),
+                                            cs))
 
     def plan_info(self) -> dict:
         pi = L.PlanInfo()
@@ -180,14 +190,22 @@ class PagedKVCache:
                 "kv_tiles": list(pi.kv_tiles[:n]), "kv_tokens": list(pi.kv_tokens[:n]),
                 "qo_len": list(pi.qo_len[:n])}
 
-    def run(self, block: int, q, out=None, lse=None, force_fp32: bool = False, cuda_stream=None):
-        """Paged attention of ``block``; returns ``out`` ([rows, H, D])."""
+    def run(self, block: int, q, out=None, lse=None, force_fp32: bool = False, cuda_stream=None,
+            k_extra=None, v_extra=None):
+        """Paged attention of ``block``; returns ``out`` ([rows, H, D]).  With
+        ``k_extra``/``v_extra`` (``svt_run_extra``) the planned dense segments are
+        attended after the pages."""
         torch = _torch()
         if out is None:
             fp32 = force_fp32 or self.dtype == "fp32"
             out = torch.empty(q.shape, dtype=torch.float32 if fp32 else q.dtype, device=q.device)
-        _check(self._lib.svt_run(self._h, block, _ptr(q), _ptr(out), _ptr(lse), int(force_fp32),
-                                 _stream_handle(cuda_stream)))
+        if k_extra is None and v_extra is None:
+            _check(self._lib.svt_run(self._h, block, _ptr(q), _ptr(out), _ptr(lse),
+                                     int(force_fp32), _stream_handle(cuda_stream)))
+        else:
+            _check(self._lib.svt_run_extra(self._h, block, _ptr(q), _ptr(k_extra), _ptr(v_extra),
+                                           _ptr(out), _ptr(lse), int(force_fp32),
+                                           _stream_handle(cuda_stream)))
         return out
 
     def frame_step(self, ks, vs, qs, outs, stream: int = 0, use_graph: bool = True,

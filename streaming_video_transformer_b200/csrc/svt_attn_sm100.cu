@@ -147,6 +147,8 @@ template <int D, bool BF16>
 __global__ void __launch_bounds__(threads_for(D), 2)
     attn_sm100_kernel(const __grid_constant__ CUtensorMap tmap_q,
                       const __grid_constant__ CUtensorMap tmap_kv,
+                      const __grid_constant__ CUtensorMap tmap_ke,
+                      const __grid_constant__ CUtensorMap tmap_ve,
                       const __grid_constant__ AttnParams p) {
   using C = Cfg<D>;
   using T = typename std::conditional<BF16, __nv_bfloat16, __half>::type;
@@ -177,6 +179,9 @@ __global__ void __launch_bounds__(threads_for(D), 2)
   const Item it = decode_item(p);
   const StreamPlan& sp = p.s[it.st];
   const int n = it.n_tiles;
+  // Tiles [0, page_tiles) of the stream come from the page table, the rest
+  // from its dense K/V segment (a frame attended without being stored).
+  const int page_tiles = sp.tiles - (sp.extra_len + TN - 1) / TN;
 
   if (threadIdx.x == 0) {
     *abort_flag = 0;
@@ -222,28 +227,46 @@ __global__ void __launch_bounds__(threads_for(D), 2)
       for (int r = 0; r < C::kRegions; ++r)
         tma_load_3d(sQ + r * C::kQRegionBytes, &tmap_q, q_full, r * 64, it.head,
                     sp.q_off + it.qtile * kTileM);
+      if (sp.extra_len > 0) {
+        tma_prefetch_desc(&tmap_ke);
+        tma_prefetch_desc(&tmap_ve);
+      }
       int issued = 0, vissued = 0;
       for (int j = 0; j < n; ++j) {
-        int page_pos, t, valid;
-        tile_coords<TN>(sp, p.P, it.t_begin + j, page_pos, t, valid);
-        int page = p.indices[sp.page_off + page_pos];
-        if (page < 0 || page >= p.max_pages) {
-          atomicOr(p.err, kErrPageId);
-          page = 0;
+        const int g = it.t_begin + j;
+        int page_pos = 0, t = 0, valid, c4 = 0, erow = 0;
+        const bool extra = g >= page_tiles;
+        if (extra) {
+          erow = sp.extra_off + (g - page_tiles) * TN;   // rows past the segment are masked
+        } else {
+          tile_coords<TN>(sp, p.P, g, page_pos, t, valid);
+          int page = p.indices[sp.page_off + page_pos];
+          if (page < 0 || page >= p.max_pages) {
+            atomicOr(p.err, kErrPageId);
+            page = 0;
+          }
+          c4 = (int)(p.block_page_base + page);
         }
-        const int c4 = (int)(p.block_page_base + page);
         const int sk = j % KS, sv = j % VS;
         if (!mbar_wait(k_empty(sk), ((j / KS) & 1) ^ 1, abort_flag, kWaitLimitNs)) { fail(); break; }
         mbar_arrive_expect_tx(k_full(sk), C::kKVBytes);
-        for (int r = 0; r < C::kRegions; ++r)
-          tma_load_5d(sK + sk * C::kKVBytes + r * C::kKVRegionBytes, &tmap_kv, k_full(sk), r * 64,
-                      it.head, t * TN, 0, c4);
+        for (int r = 0; r < C::kRegions; ++r) {
+          const uint32_t dst = sK + sk * C::kKVBytes + r * C::kKVRegionBytes;
+          if (extra)
+            tma_load_3d(dst, &tmap_ke, k_full(sk), r * 64, it.head, erow);
+          else
+            tma_load_5d(dst, &tmap_kv, k_full(sk), r * 64, it.head, t * TN, 0, c4);
+        }
         issued = j + 1;
         if (!mbar_wait(v_empty(sv), ((j / VS) & 1) ^ 1, abort_flag, kWaitLimitNs)) { fail(); break; }
         mbar_arrive_expect_tx(v_full(sv), C::kKVBytes);
-        for (int r = 0; r < C::kRegions; ++r)
-          tma_load_5d(sV + sv * C::kKVBytes + r * C::kKVRegionBytes, &tmap_kv, v_full(sv), r * 64,
-                      it.head, t * TN, 1, c4);
+        for (int r = 0; r < C::kRegions; ++r) {
+          const uint32_t dst = sV + sv * C::kKVBytes + r * C::kKVRegionBytes;
+          if (extra)
+            tma_load_3d(dst, &tmap_ve, v_full(sv), r * 64, it.head, erow);
+          else
+            tma_load_5d(dst, &tmap_kv, v_full(sv), r * 64, it.head, t * TN, 1, c4);
+        }
         vissued = j + 1;
       }
       if (*abort_flag) {
@@ -330,10 +353,14 @@ __global__ void __launch_bounds__(threads_for(D), 2)
     int page_pos, t, valid;
     tile_coords<TN>(sp, P, it.t_begin, page_pos, t, valid);
     for (int j = 0; j < n && ok; ++j) {
-      valid = min(TN, (page_pos < last_page ? P : lpl) - t * TN);
-      if (++t == tpp && page_pos < last_page) {
-        t = 0;
-        ++page_pos;
+      if (it.t_begin + j < page_tiles) {
+        valid = min(TN, (page_pos < last_page ? P : lpl) - t * TN);
+        if (++t == tpp && page_pos < last_page) {
+          t = 0;
+          ++page_pos;
+        }
+      } else {
+        valid = min(TN, sp.extra_len - (it.t_begin + j - page_tiles) * TN);
       }
       ok = __all_sync(kAll, mbar_wait(s_full, j & 1, abort_flag, kWaitLimitNs));
       if (!ok) break;
@@ -514,8 +541,8 @@ __global__ void __launch_bounds__(threads_for(D), 2)
 }
 
 template <int D, bool BF16>
-cudaError_t launch_t(const AttnParams& p, const void* tq, const void* tkv, cudaStream_t s,
-                     Recorder* rec) {
+cudaError_t launch_t(const AttnParams& p, const void* tq, const void* tkv, const void* tke,
+                     const void* tve, cudaStream_t s, Recorder* rec) {
   using C = Cfg<D>;
   auto kern = attn_sm100_kernel<D, BF16>;
   static bool configured = false;
@@ -525,10 +552,13 @@ cudaError_t launch_t(const AttnParams& p, const void* tq, const void* tkv, cudaS
     if (e != cudaSuccess) return e;
     configured = true;
   }
-  CUtensorMap mq, mkv;
+  CUtensorMap mq, mkv, mke, mve;
   memcpy(&mq, tq, sizeof(mq));
   memcpy(&mkv, tkv, sizeof(mkv));
-  return dispatch(rec, kern, p.total_items, threads_for(D), C::kSmemBytes, s, mq, mkv, p);
+  memcpy(&mke, tke ? tke : tq, sizeof(mke));
+  memcpy(&mve, tve ? tve : tq, sizeof(mve));
+  return dispatch(rec, kern, p.total_items, threads_for(D), C::kSmemBytes, s, mq, mkv, mke, mve,
+                  p);
 }
 
 
@@ -542,13 +572,16 @@ int attn_items_per_stream(int H, int D, int qtiles, int chunks) {
 int attn_ctas_per_sm(int D) { (void)D; return 2; }   // 256 TMEM columns and < 113 KB smem each
 
 cudaError_t launch_attn_sm100(const AttnParams& p, const void* tmap_q, const void* tmap_kv,
-                              int dtype, cudaStream_t s, Recorder* rec) {
+                              const void* tmap_ke, const void* tmap_ve, int dtype,
+                              cudaStream_t s, Recorder* rec) {
   if (p.total_items == 0) return cudaSuccess;
   const bool bf16 = dtype == SVT_BF16;
-  if (p.D == 64) return bf16 ? launch_t<64, true>(p, tmap_q, tmap_kv, s, rec)
-                             : launch_t<64, false>(p, tmap_q, tmap_kv, s, rec);
-  if (p.D == 128) return bf16 ? launch_t<128, true>(p, tmap_q, tmap_kv, s, rec)
-                              : launch_t<128, false>(p, tmap_q, tmap_kv, s, rec);
+  if (p.D == 64)
+    return bf16 ? launch_t<64, true>(p, tmap_q, tmap_kv, tmap_ke, tmap_ve, s, rec)
+                : launch_t<64, false>(p, tmap_q, tmap_kv, tmap_ke, tmap_ve, s, rec);
+  if (p.D == 128)
+    return bf16 ? launch_t<128, true>(p, tmap_q, tmap_kv, tmap_ke, tmap_ve, s, rec)
+                : launch_t<128, false>(p, tmap_q, tmap_kv, tmap_ke, tmap_ve, s, rec);
   return cudaErrorInvalidValue;
 }
 

@@ -124,6 +124,7 @@ struct svt_cache {
   bool plan_valid = false;
   uint64_t plan_version = 0;
   int total_rows = 0;
+  int extra_rows = 0;      // rows of the dense K/V segments of the plan
   bool any_split = false;
   AttnParams attn{};
   SimtParams simt{};
@@ -141,6 +142,7 @@ struct svt_cache {
   float* d_ws_o = nullptr;
   float* d_ws_lse = nullptr;
   char* d_qrope = nullptr;
+  char* d_krope = nullptr;     // RoPE'd K of the dense segments
   float2* d_rope_tab = nullptr;
   int ring_cap = 1, sp_cap = 0, indices_cap = 0;
 
@@ -149,6 +151,7 @@ struct svt_cache {
   alignas(64) CUtensorMap tmap_q;
   const void* tmap_q_ptr = nullptr;
   int tmap_q_rows = -1;
+  alignas(64) CUtensorMap tmap_ke, tmap_ve;   // dense K/V segments (box of TN rows)
 
   // frame steps replayed as CUDA graphs (svt_frame_step): the launches of a
   // step are recorded into `rec` instead of being issued, then handed to an
@@ -222,22 +225,29 @@ int encode_kv_map(svt_cache* c) {
   return SVT_OK;
 }
 
-int encode_q_map(svt_cache* c, const void* q, int rows) {
-  if (c->tmap_q_ptr == q && c->tmap_q_rows == rows) return SVT_OK;
+// Tensor map over a dense [rows][H][D] array with boxes of box_rows rows.
+int encode_rows_map(const svt_cache* c, CUtensorMap* map, const void* base, int rows,
+                    int box_rows, const char* what) {
   auto enc = tensor_map_encoder();
   if (!enc) return fail(SVT_ECUDA, "cuTensorMapEncodeTiled entry point unavailable");
   const cuuint64_t e = c->elem;
   cuuint64_t dims[3] = {(cuuint64_t)c->D, (cuuint64_t)c->H, (cuuint64_t)rows};
   cuuint64_t strides[2] = {c->D * e, (cuuint64_t)c->H * c->D * e};
-  cuuint32_t box[3] = {64, 1, (cuuint32_t)kTileM};
+  cuuint32_t box[3] = {64, 1, (cuuint32_t)box_rows};
   cuuint32_t estr[3] = {1, 1, 1};
-  CUresult r = enc(&c->tmap_q,
+  CUresult r = enc(map,
                    c->dtype == SVT_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16
                                         : CU_TENSOR_MAP_DATA_TYPE_FLOAT16,
-                   3, const_cast<void*>(q), dims, strides, box, estr,
+                   3, const_cast<void*>(base), dims, strides, box, estr,
                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-  if (r != CUDA_SUCCESS) return fail(SVT_ECUDA, "cuTensorMapEncodeTiled(q) failed: %d", (int)r);
+  if (r != CUDA_SUCCESS) return fail(SVT_ECUDA, "cuTensorMapEncodeTiled(%s) failed: %d", what, (int)r);
+  return SVT_OK;
+}
+
+int encode_q_map(svt_cache* c, const void* q, int rows) {
+  if (c->tmap_q_ptr == q && c->tmap_q_rows == rows) return SVT_OK;
+  if (int r = encode_rows_map(c, &c->tmap_q, q, rows, kTileM, "q")) return r;
   c->tmap_q_ptr = q;
   c->tmap_q_rows = rows;
   return SVT_OK;
@@ -426,6 +436,7 @@ int svt_create_cache(int max_pages, int page_size, int H, int D, int sliding_win
     size_t o_ws_o = carve(sizeof(float) * (size_t)c->max_splits * c->max_qo * H * D);
     size_t o_ws_lse = carve(sizeof(float) * (size_t)c->max_splits * c->max_qo * H);
     size_t o_qrope = c->rope_grid ? carve((size_t)c->max_qo * H * D * c->elem) : 0;
+    size_t o_krope = c->rope_grid ? carve((size_t)c->max_qo * H * D * c->elem) : 0;
     std::vector<float2> tab;
     if (c->rope_grid) fill_rope_table(c, tab);
     size_t o_tab = c->rope_grid ? carve(sizeof(float2) * tab.size()) : 0;
@@ -443,6 +454,7 @@ int svt_create_cache(int max_pages, int page_size, int H, int D, int sliding_win
     c->d_ws_lse = reinterpret_cast<float*>(b + o_ws_lse);
     if (c->rope_grid) {
       c->d_qrope = b + o_qrope;
+      c->d_krope = b + o_krope;
       c->d_rope_tab = reinterpret_cast<float2*>(b + o_tab);
     }
     e = cudaMemset(c->dmem, 0, off);
@@ -765,7 +777,11 @@ int svt_read_device_page_table(svt_cache* c, int32_t* indptr, int32_t* indices,
   return SVT_OK;
 }
 
-int svt_plan(svt_cache* c, const int32_t* qo_len, svt_stream_t) {
+int svt_plan(svt_cache* c, const int32_t* qo_len, svt_stream_t s) {
+  return svt_plan_extra(c, qo_len, nullptr, s);
+}
+
+int svt_plan_extra(svt_cache* c, const int32_t* qo_len, const int32_t* extra_len, svt_stream_t) {
   if (!c) return fail(SVT_EINVAL, "null cache");
   if (!qo_len) return fail(SVT_EINVAL, "qo_len_per_stream is NULL");
   if (c->dirty) return fail(SVT_ESTATE, "cache changed since build_visible_page_table");
@@ -781,12 +797,18 @@ int svt_plan(svt_cache* c, const int32_t* qo_len, svt_stream_t) {
   svt_plan_info& info = c->info;
   info = svt_plan_info{};
   std::vector<int> tiles(c->n_streams, 0), qt(c->n_streams, 0);
+  int extra_rows = 0;
   for (int i = 0; i < c->n_streams; ++i) {
     const StreamState& s = c->st[i];
     const int np = n_visible_pages(s);
     const int lpl = page_valid_tokens_last(c, s);
-    if (qo_len[i] < 0) return fail(SVT_EINVAL, "negative qo_len");
-    if (qo_len[i] > 0 && np == 0)
+    const int xl = extra_len ? extra_len[i] : 0;
+    if (qo_len[i] < 0 || xl < 0) return fail(SVT_EINVAL, "negative qo_len or extra_len");
+    if (xl > 0 && qo_len[i] == 0) return fail(SVT_EINVAL, "stream %d: extra_len without queries", i);
+    if (c->rope_grid && xl % (c->ns + P))
+      return fail(SVT_EINVAL, "with RoPE each stream's extra segment is whole frames of %d rows",
+                  c->ns + P);
+    if (qo_len[i] > 0 && np == 0 && xl == 0)
       return fail(SVT_ESTATE, "stream %d has queries but no visible tokens", i);
     if (c->rope_grid && qo_len[i] % (c->ns + P))
       return fail(SVT_EINVAL, "with RoPE each stream's query is whole frames of %d rows", c->ns + P);
@@ -797,16 +819,21 @@ int svt_plan(svt_cache* c, const int32_t* qo_len, svt_stream_t) {
     sp.page_off = page_off;
     sp.n_pages = np;
     sp.lpl = lpl;
-    sp.tiles = np ? (np - 1) * tpp + (lpl + TN - 1) / TN : 0;
+    sp.tiles = (np ? (np - 1) * tpp + (lpl + TN - 1) / TN : 0) + (xl + TN - 1) / TN;
+    sp.extra_len = xl;
+    sp.extra_off = extra_rows;
+    extra_rows += xl;
     tiles[i] = sp.tiles;
     qt[i] = sp.qtiles;
     rows += qo_len[i];
     page_off += np;
     info.kv_tiles[i] = sp.tiles;
-    info.kv_tokens[i] = np ? (int64_t)(np - 1) * PT + lpl : 0;
+    info.kv_tokens[i] = (np ? (int64_t)(np - 1) * PT + lpl : 0) + xl;
     info.qo_len[i] = qo_len[i];
   }
   if (rows > c->max_qo) return fail(SVT_EINVAL, "total query rows %d > max_qo_len %d", rows, c->max_qo);
+  if (extra_rows > c->max_qo)
+    return fail(SVT_EINVAL, "total extra rows %d > max_qo_len %d", extra_rows, c->max_qo);
   // Choose KV splits: candidate k scales every stream's chunk count with its tile count.
   int max_tiles = 0;
   for (int i = 0; i < c->n_streams; ++i)
@@ -886,6 +913,8 @@ int svt_plan(svt_cache* c, const int32_t* qo_len, svt_stream_t) {
     ss.page_off = a.s[i].page_off;
     ss.n_pages = a.s[i].n_pages;
     ss.lpl = a.s[i].lpl;
+    ss.extra_len = a.s[i].extra_len;
+    ss.extra_off = a.s[i].extra_off;
     ss.block_off = blocks;
     blocks += ss.rblocks * c->H;
   }
@@ -898,6 +927,7 @@ int svt_plan(svt_cache* c, const int32_t* qo_len, svt_stream_t) {
   m.scale = (float)(1.0 / std::sqrt((double)c->D));
   m.err = c->d_err;
   c->total_rows = rows;
+  c->extra_rows = extra_rows;
   c->any_split = any_split;
   c->plan_valid = true;
   c->plan_version = c->version;
@@ -913,6 +943,11 @@ int svt_get_plan_info(const svt_cache* c, svt_plan_info* out) {
 
 int svt_run(svt_cache* c, int block, const void* q, void* out, float* lse, int force_fp32,
             svt_stream_t cs) {
+  return svt_run_extra(c, block, q, nullptr, nullptr, out, lse, force_fp32, cs);
+}
+
+int svt_run_extra(svt_cache* c, int block, const void* q, const void* k_extra,
+                  const void* v_extra, void* out, float* lse, int force_fp32, svt_stream_t cs) {
   if (!c) return fail(SVT_EINVAL, "null cache");
   if (c->host_only) return fail(SVT_EINVAL, "host-only cache cannot run kernels");
   if (block < 0 || block >= c->L) return fail(SVT_EINVAL, "block %d out of range", block);
@@ -920,11 +955,16 @@ int svt_run(svt_cache* c, int block, const void* q, void* out, float* lse, int f
     return fail(SVT_ESTATE, "no valid plan for the current page table (build, then plan)");
   if (c->total_rows == 0) return SVT_OK;
   if (!q || !out) return fail(SVT_EINVAL, "q and out must be device pointers");
+  if (c->extra_rows > 0 && (!k_extra || !v_extra))
+    return fail(SVT_EINVAL, "the plan has dense K/V segments: pass k_extra and v_extra");
+  if (c->extra_rows == 0 && (k_extra || v_extra))
+    return fail(SVT_EINVAL, "the plan has no dense K/V segment (plan with extra_len)");
   for (int i = 0; i < c->n_streams; ++i)
-    if (c->attn.s[i].nq && c->st[i].blocks_done <= block)
+    if (c->attn.s[i].nq && c->attn.s[i].extra_len == 0 && c->st[i].blocks_done <= block)
       return fail(SVT_ESTATE, "stream %d: block %d has not appended the current frame", i, block);
   cudaStream_t s = reinterpret_cast<cudaStream_t>(cs);
   const char* qsrc = static_cast<const char*>(q);
+  const char* ksrc = static_cast<const char*>(k_extra);
   cudaError_t e;
   if (c->rope_grid) {
     RopeQParams rp{};
@@ -941,12 +981,22 @@ int svt_run(svt_cache* c, int block, const void* q, void* out, float* lse, int f
     e = launch_rope_q(rp, c->dtype, s, c->rec);
     if (e != cudaSuccess) return cuda_fail(e, "rope_q launch");
     qsrc = c->d_qrope;
+    if (c->extra_rows > 0) {   // the segment's K gets the same rotation as stored keys
+      rp.q_in = ksrc;
+      rp.q_out = c->d_krope;
+      rp.rows = c->extra_rows;
+      e = launch_rope_q(rp, c->dtype, s, c->rec);
+      if (e != cudaSuccess) return cuda_fail(e, "rope_k launch");
+      ksrc = c->d_krope;
+    }
   }
   const size_t block_bytes = (size_t)c->max_pages * 2 * c->page_tokens * c->H * c->D * c->elem;
   if (force_fp32 || c->dtype == SVT_FP32) {
     SimtParams m = c->simt;
     m.pool_block = c->pool + (size_t)block * block_bytes;
     m.q = qsrc;
+    m.k_extra = ksrc;
+    m.v_extra = static_cast<const char*>(v_extra);
     m.out = static_cast<float*>(out);
     m.lse = lse;
     e = launch_attn_simt(m, c->dtype, s, c->rec);
@@ -955,11 +1005,19 @@ int svt_run(svt_cache* c, int block, const void* q, void* out, float* lse, int f
   }
   if (reinterpret_cast<uintptr_t>(qsrc) % 16) return fail(SVT_EINVAL, "q must be 16-byte aligned");
   if (int r = encode_q_map(c, qsrc, c->total_rows)) return r;
+  if (c->extra_rows > 0) {
+    if ((reinterpret_cast<uintptr_t>(ksrc) | reinterpret_cast<uintptr_t>(v_extra)) % 16)
+      return fail(SVT_EINVAL, "k_extra and v_extra must be 16-byte aligned");
+    const int tn = attn_tile_n(c->D);
+    if (int r = encode_rows_map(c, &c->tmap_ke, ksrc, c->extra_rows, tn, "k_extra")) return r;
+    if (int r = encode_rows_map(c, &c->tmap_ve, v_extra, c->extra_rows, tn, "v_extra")) return r;
+  }
   AttnParams a = c->attn;
   a.block_page_base = (int64_t)block * c->max_pages;
   a.out = out;
   a.lse = lse;
-  e = launch_attn_sm100(a, &c->tmap_q, &c->tmap_kv, c->dtype, s, c->rec);
+  e = launch_attn_sm100(a, &c->tmap_q, &c->tmap_kv, c->extra_rows ? &c->tmap_ke : nullptr,
+                        c->extra_rows ? &c->tmap_ve : nullptr, c->dtype, s, c->rec);
   if (e != cudaSuccess) return cuda_fail(e, "attention launch");
   if (c->any_split) {
     e = launch_merge(a, c->dtype, s, c->rec);

@@ -149,8 +149,11 @@ struct StreamPlan {
   int page_off;     // first entry of the stream in the visible table
   int n_pages;      // entries in the visible table
   int lpl;          // valid tokens on the last page
-  int tiles;        // KV tiles: (n_pages-1)*ceil(P/TN) + ceil(lpl/TN), TN = attn_tile_n(D)
+  int tiles;        // KV tiles: (n_pages-1)*ceil(P/TN) + ceil(lpl/TN) + ceil(extra_len/TN),
+                    // TN = attn_tile_n(D)
   int item_off;     // first work item of the stream
+  int extra_len;    // rows of a dense K/V segment attended after the pages (0 = none)
+  int extra_off;    // first row of the stream's segment in the dense K/V arrays
 };
 
 struct AttnParams {
@@ -170,22 +173,27 @@ struct AttnParams {
 
 // Tensor-core (tcgen05 / TMEM) kernel; tensor maps are CUtensorMap (128 bytes each).
 // One work item covers one 128-row query tile of one (stream, head, KV chunk).
+// tmap_ke / tmap_ve map the dense K/V segments (box of TN rows); they are only
+// read for streams with extra_len > 0 and may repeat another map otherwise.
 int attn_items_per_stream(int H, int D, int qtiles, int chunks);
 int attn_ctas_per_sm(int D);   // resident CTAs of the tensor-core kernel per SM
 cudaError_t launch_attn_sm100(const AttnParams& p, const void* tmap_q, const void* tmap_kv,
-                              int dtype, cudaStream_t s, Recorder* rec);
+                              const void* tmap_ke, const void* tmap_ve, int dtype,
+                              cudaStream_t s, Recorder* rec);
 
 // Combines split-KV partials into out / lse.
 cudaError_t launch_merge(const AttnParams& p, int dtype, cudaStream_t s, Recorder* rec);
 
 // fp32-FMA kernel (force_fp32 / fp32 pool).  Writes fp32 out and lse directly.
-struct SimtStream { int q_off, nq, rblocks, page_off, n_pages, lpl, block_off; };
+struct SimtStream { int q_off, nq, rblocks, page_off, n_pages, lpl, block_off, extra_len, extra_off; };
 struct SimtParams {
   int n_streams, total_blocks;
   int H, D, P, max_pages;    // P = tokens per pool page
   const char* pool_block;
   const int* indices;
   const char* q;
+  const char* k_extra;       // dense K/V segments [rows][H][D] (nullptr when none)
+  const char* v_extra;
   float* out;
   float* lse;
   float scale;               // 1 / sqrt(D)

@@ -262,6 +262,62 @@ __global__ void __launch_bounds__(kSimtThreads) attn_simt_kernel(SimtParams p) {
   }
   float m = -INFINITY, l = 0.f, lc = 0.f;
   const T* pool = reinterpret_cast<const T*>(p.pool_block);
+  // One tile of nt <= kSimtKT tokens whose K and V rows start at kt and vt
+  // (row stride H*D): stage it, score it and fold it into (m, l, o).
+  auto tile = [&](const T* kt, const T* vt, int nt) {
+    __syncthreads();
+    for (int e = threadIdx.x; e < kSimtKT * D; e += kSimtThreads) {
+      const int j = e / D, d = e % D;
+      float kx = 0.f, vx = 0.f;
+      if (j < nt) {
+        kx = to_f(kt[(size_t)j * HD + d]);
+        vx = to_f(vt[(size_t)j * HD + d]);
+      }
+      ks[j][d / 32][d % 32] = kx;
+      vs[j][d / 32][d % 32] = vx;
+    }
+    __syncthreads();
+    float s[kSimtKT];
+    float tmax = -INFINITY;
+#pragma unroll
+    for (int j = 0; j < kSimtKT; ++j) {
+      float acc = 0.f;
+#pragma unroll
+      for (int i = 0; i < 32; ++i) acc = fmaf(q[i], ks[j][part][i], acc);
+#pragma unroll
+      for (int w = 1; w < TPR; w <<= 1) acc += __shfl_xor_sync(0xffffffffu, acc, w);
+      s[j] = j < nt ? acc * p.scale : -INFINITY;
+      tmax = fmaxf(tmax, s[j]);
+    }
+    const float mnew = fmaxf(m, tmax);
+    const float alpha = expf(m - mnew);   // m = -inf on the first tile -> 0
+    m = mnew;
+    float ot[32], lt = 0.f;
+#pragma unroll
+    for (int i = 0; i < 32; ++i) ot[i] = 0.f;
+#pragma unroll
+    for (int j = 0; j < kSimtKT; ++j) {
+      const float pj = expf(s[j] - m);
+      lt += pj;
+#pragma unroll
+      for (int i = 0; i < 32; ++i) ot[i] = fmaf(pj, vs[j][part][i], ot[i]);
+    }
+    {
+      const float lr = __fmul_rn(l, alpha), lcr = __fmul_rn(lc, alpha);
+      const float y = __fsub_rn(lt, lcr);
+      const float tt = __fadd_rn(lr, y);
+      lc = __fsub_rn(__fsub_rn(tt, lr), y);
+      l = tt;
+    }
+#pragma unroll
+    for (int i = 0; i < 32; ++i) {
+      const float orr = __fmul_rn(o[i], alpha), ocr = __fmul_rn(oc[i], alpha);
+      const float y = __fsub_rn(ot[i], ocr);
+      const float tt = __fadd_rn(orr, y);
+      oc[i] = __fsub_rn(__fsub_rn(tt, orr), y);
+      o[i] = tt;
+    }
+  };
   for (int pp = 0; pp < S.n_pages; ++pp) {
     int page = p.indices[S.page_off + pp];
     if (page < 0 || page >= p.max_pages) {
@@ -271,61 +327,15 @@ __global__ void __launch_bounds__(kSimtThreads) attn_simt_kernel(SimtParams p) {
     const int valid = pp == S.n_pages - 1 ? S.lpl : p.P;
     const T* kpage = pool + (size_t)page * 2 * p.P * HD + h * D;
     const T* vpage = kpage + (size_t)p.P * HD;
-    for (int t0 = 0; t0 < valid; t0 += kSimtKT) {
-      const int nt = min(kSimtKT, valid - t0);
-      __syncthreads();
-      for (int e = threadIdx.x; e < kSimtKT * D; e += kSimtThreads) {
-        const int j = e / D, d = e % D;
-        float kx = 0.f, vx = 0.f;
-        if (j < nt) {
-          kx = to_f(kpage[(size_t)(t0 + j) * HD + d]);
-          vx = to_f(vpage[(size_t)(t0 + j) * HD + d]);
-        }
-        ks[j][d / 32][d % 32] = kx;
-        vs[j][d / 32][d % 32] = vx;
-      }
-      __syncthreads();
-      float s[kSimtKT];
-      float tmax = -INFINITY;
-#pragma unroll
-      for (int j = 0; j < kSimtKT; ++j) {
-        float acc = 0.f;
-#pragma unroll
-        for (int i = 0; i < 32; ++i) acc = fmaf(q[i], ks[j][part][i], acc);
-#pragma unroll
-        for (int w = 1; w < TPR; w <<= 1) acc += __shfl_xor_sync(0xffffffffu, acc, w);
-        s[j] = j < nt ? acc * p.scale : -INFINITY;
-        tmax = fmaxf(tmax, s[j]);
-      }
-      const float mnew = fmaxf(m, tmax);
-      const float alpha = expf(m - mnew);   // m = -inf on the first tile -> 0
-      m = mnew;
-      float ot[32], lt = 0.f;
-#pragma unroll
-      for (int i = 0; i < 32; ++i) ot[i] = 0.f;
-#pragma unroll
-      for (int j = 0; j < kSimtKT; ++j) {
-        const float pj = expf(s[j] - m);
-        lt += pj;
-#pragma unroll
-        for (int i = 0; i < 32; ++i) ot[i] = fmaf(pj, vs[j][part][i], ot[i]);
-      }
-      {
-        const float lr = __fmul_rn(l, alpha), lcr = __fmul_rn(lc, alpha);
-        const float y = __fsub_rn(lt, lcr);
-        const float tt = __fadd_rn(lr, y);
-        lc = __fsub_rn(__fsub_rn(tt, lr), y);
-        l = tt;
-      }
-#pragma unroll
-      for (int i = 0; i < 32; ++i) {
-        const float orr = __fmul_rn(o[i], alpha), ocr = __fmul_rn(oc[i], alpha);
-        const float y = __fsub_rn(ot[i], ocr);
-        const float tt = __fadd_rn(orr, y);
-        oc[i] = __fsub_rn(__fsub_rn(tt, orr), y);
-        o[i] = tt;
-      }
-    }
+    for (int t0 = 0; t0 < valid; t0 += kSimtKT)
+      tile(kpage + (size_t)t0 * HD, vpage + (size_t)t0 * HD, min(kSimtKT, valid - t0));
+  }
+  // The stream's dense K/V segment (a frame attended without being stored).
+  if (S.extra_len > 0) {
+    const T* ke = reinterpret_cast<const T*>(p.k_extra) + (size_t)S.extra_off * HD + h * D;
+    const T* ve = reinterpret_cast<const T*>(p.v_extra) + (size_t)S.extra_off * HD + h * D;
+    for (int t0 = 0; t0 < S.extra_len; t0 += kSimtKT)
+      tile(ke + (size_t)t0 * HD, ve + (size_t)t0 * HD, min(kSimtKT, S.extra_len - t0));
   }
   if (!active) return;
   const float inv = 1.f / l;

@@ -216,7 +216,7 @@ extern "C" SVT_API int svt_attention_noalloc(
       return err(SVT_ECUDA, "cuTensorMapEncodeTiled(pool) failed");
   }
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  cudaError_t e = launch_attn_sm100(a, &tq, &tkv, dtype, s, nullptr);
+  cudaError_t e = launch_attn_sm100(a, &tq, &tkv, nullptr, nullptr, dtype, s, nullptr);
   if (e != cudaSuccess) return err(SVT_ECUDA, "attention launch: %s", cudaGetErrorString(e));
   if (splits > 1) {
     e = launch_merge(a, dtype, s, nullptr);

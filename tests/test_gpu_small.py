@@ -8,6 +8,7 @@ import golden_io
 from alloc_model import AllocModel
 from gpu_util import (FrameBank, assert_close, gather_visible, make_cache, max_pages_for,
                       oracle_out, oracle_stream)
+from oracle import attend_lse
 from streaming_video_transformer_b200.inputs import WORKLOADS, frame_qkv, small_workload
 
 pytestmark = pytest.mark.gpu
@@ -329,4 +330,71 @@ def test_row_max_jumps_in_later_tiles(dtype, jump, splits):
     assert_close(out, ref, what=f"{dtype} jump {jump}")
     np.testing.assert_allclose(lse.cpu().numpy(), lse_ref, rtol=1e-3, atol=2e-2)
     assert_close(c.run(0, q.cuda(), force_fp32=True), ref, fp32=True, what=f"fp32 jump {jump}")
+    c.device_error()
+
+
+SEGMENT = [
+    dict(P=48, ns=6, S=2, W=3, H=2, D=64),                         # bf16
+    dict(P=36, ns=6, S=1, W=2, H=2, D=64, rope_grid=6),            # 2-D RoPE on the segment's K
+    dict(P=100, ns=6, S=1, W=3, H=2, D=128, dtype="fp16"),         # 64-token tiles, ragged tail
+]
+
+
+@pytest.mark.parametrize("cfg", SEGMENT, ids=[str(i) for i in range(len(SEGMENT))])
+def test_skip_append_with_dense_segment(cfg):
+    """A non-keyframe attends to the cache plus its own K/V given as a dense
+    segment: nothing is written to the pool and the allocator is untouched.
+    Stream 0 attends with its frame as a segment, stream 1 (in the same run)
+    with its cache only."""
+    w = small_workload(**cfg, R=16)
+    c = make_cache(w, max_pages_for(w, [12, 12], num_streams=2), num_streams=2)
+    banks = [FrameBank(w, 0, s) for s in range(2)]
+    sts = [oracle_stream(w) for _ in range(2)]
+    for s in range(2):
+        for t in range(7):
+            c.append_frame(0, *banks[s].device(t)[1:], stream=s)
+            c.evict_frames(s)
+            sts[s].append_frame(*banks[s].oracle(t)[1:])
+    c.build_visible_page_table()
+    table, stats = c.get_page_table(), c.get_cache_stats()
+    pool0 = c.pool.clone()
+    q7, k7, v7 = banks[0].device(7)
+    q1 = banks[1].device(6)[0]
+    c.plan([w.Nq, w.Nq], extra_len=[w.Nq, 0])
+    info = c.plan_info()
+    assert info["kv_tokens"][0] == sts[0].num_visible_tokens() + w.Nq
+    q = torch.cat([q7, q1])
+    out = c.run(0, q, k_extra=k7, v_extra=v7)
+    out32 = c.run(0, q, k_extra=k7, v_extra=v7, force_fp32=True)
+    q64, k64, v64 = banks[0].oracle(7)
+    kc, vc = sts[0].visible_kv()
+    ref0, _ = attend_lse(q64, np.concatenate([kc, k64]), np.concatenate([vc, v64]))
+    ref1, _ = oracle_out(sts[1], banks[1].oracle(6)[0])
+    assert_close(out[:w.Nq], ref0, what="segment stream")
+    assert_close(out32[:w.Nq], ref0, fp32=True, what="segment stream fp32")
+    assert_close(out[w.Nq:], ref1, what="plain stream")
+    assert_close(out32[w.Nq:], ref1, fp32=True, what="plain stream fp32")
+    # nothing stored, nothing allocated
+    assert torch.equal(c.pool, pool0)
+    for a, b in zip(table, c.get_page_table()):
+        assert np.array_equal(a, b)
+    assert c.get_cache_stats() == stats
+    # the deferred append / attend / rollback route gives the same attention
+    c.set_defer_eviction(True, 0)
+    c.append_frame(0, k7, v7, stream=0)
+    c.evict_frames(0)
+    c.build_visible_page_table()
+    c.plan([w.Nq, 0])
+    via_pool = c.run(0, q7)
+    assert_close(via_pool, out[:w.Nq].double().cpu().numpy(), what="segment vs deferred append")
+    c.rollback_last_frame(0)
+    c.set_defer_eviction(False, 0)
+    # the next stored frame sees exactly the cache it would have seen
+    c.append_frame(0, *banks[0].device(8)[1:], stream=0)
+    c.evict_frames(0)
+    sts[0].append_frame(*banks[0].oracle(8)[1:])
+    c.build_visible_page_table()
+    c.plan([w.Nq, 0])
+    ref, _ = oracle_out(sts[0], banks[0].oracle(8)[0])
+    assert_close(c.run(0, banks[0].device(8)[0]), ref, what="frame after the segment step")
     c.device_error()

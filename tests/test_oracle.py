@@ -351,3 +351,26 @@ def test_rope_dot_product_depends_only_on_offset():
         d1 = RX[r1 * grid + c1, 0] @ RY[r2 * grid + c2, 0]
         d2 = RX[(r1 + 1) * grid + c1 - 0, 0] @ RY[(r2 + 1) * grid + c2, 0] if r2 + 1 < grid else d1
         assert abs(d1 - d2) < 1e-5
+
+
+def test_deferred_frame_visible_set_is_cache_plus_the_frame():
+    """Attending a frame without storing it (cache + the frame's own rows)
+    sees the same tokens as appending it with eviction deferred: compared
+    as sets of rows, with and without special retention."""
+    rng = np.random.default_rng(12)
+    for cross in (True, False):
+        for S, W in ((2, 3), (0, 2), (3, 1), (1, 0)):
+            st = FrameStream(3, 2, S, W, cross_frame_special=cross)
+            for t in range(7):
+                k = rng.standard_normal((5, 1, 4))
+                st.append_frame(k, k + 1.0)
+                kf = rng.standard_normal((5, 1, 4))
+                vf = kf + 1.0
+                kc, vc = st.visible_kv()
+                plus = np.concatenate([kc, kf])
+                st.append_frame(kf, vf, deferred=True)
+                kd, _ = st.visible_kv()
+                st.rollback_last_frame()
+                a = sorted(map(tuple, plus.reshape(len(plus), -1)))
+                b = sorted(map(tuple, kd.reshape(len(kd), -1)))
+                assert a == b, (cross, S, W, t)
