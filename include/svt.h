@@ -265,8 +265,10 @@ SVT_API int svt_run_extra(svt_cache* c, int block, const void* q, const void* k_
  * use_graph = 1: the step's launches are recorded and issued as one CUDA graph launch.  The
  * library keeps an executable graph per launch sequence met (up to 8): the first step with a
  * new sequence builds and instantiates it, later steps give its kernel nodes the new arguments
- * (page ids, plan) and relaunch it.  Results are bit-identical to use_graph = 0.  The graphs
- * live until svt_destroy_cache; calls on one cache must come from one host thread.
+ * (page ids, plan) and relaunch it (a graph that refuses the new arguments is rebuilt; if no
+ * graph can be built the step is launched kernel by kernel).  Results are bit-identical to
+ * use_graph = 0.  svt_get_graph_counts reports builds and replays.  The graphs live until
+ * svt_destroy_cache; calls on one cache must come from one host thread.
  * Errors: as the calls it makes; the host bookkeeping of the sub-steps that succeeded stands
  * and their kernels are issued. */
 SVT_API int svt_frame_step(svt_cache* c, int stream, const void* const* k, const void* const* v,

@@ -1076,17 +1076,22 @@ int svt_frame_step(svt_cache* c, int stream, const void* const* k, const void* c
     if (x.funcs == funcs) g = &x;
   std::vector<void*> argv;
   if (g) {
-    for (size_t i = 0; i < rec.launches.size(); ++i) {
+    bool updated = true;
+    for (size_t i = 0; updated && i < rec.launches.size(); ++i) {
       cudaKernelNodeParams kp = node_params(rec.launches[i], argv);
-      cudaError_t e = cudaGraphExecKernelNodeSetParams(g->exec, g->nodes[i], &kp);
-      if (e != cudaSuccess) {
-        cudaGetLastError();
-        issue_directly(rec, s);
-        return cuda_fail(e, "graph node update");
-      }
+      updated = cudaGraphExecKernelNodeSetParams(g->exec, g->nodes[i], &kp) == cudaSuccess;
     }
-    c->graph_replays += 1;
-  } else {
+    if (updated) {
+      c->graph_replays += 1;
+    } else {                         // the executable graph refused the new arguments: rebuild it
+      cudaGetLastError();
+      cudaGraphExecDestroy(g->exec);
+      cudaGraphDestroy(g->graph);
+      c->graphs.erase(c->graphs.begin() + (g - c->graphs.data()));
+      g = nullptr;
+    }
+  }
+  if (!g) {
     if (c->graphs.size() >= 8) {     // keep a few launch sequences
       cudaGraphExecDestroy(c->graphs.front().exec);
       cudaGraphDestroy(c->graphs.front().graph);
@@ -1104,11 +1109,11 @@ int svt_frame_step(svt_cache* c, int stream, const void* const* k, const void* c
       prev = node;
     }
     if (e == cudaSuccess) e = cudaGraphInstantiate(&ng.exec, ng.graph, 0);
-    if (e != cudaSuccess) {
+    if (e != cudaSuccess) {          // no graph: the step still runs, launch by launch
       if (ng.graph) cudaGraphDestroy(ng.graph);
       cudaGetLastError();
-      issue_directly(rec, s);
-      return cuda_fail(e, "graph build");
+      e = issue_directly(rec, s);
+      return e == cudaSuccess ? SVT_OK : cuda_fail(e, "frame step launches");
     }
     c->graphs.push_back(std::move(ng));
     g = &c->graphs.back();
