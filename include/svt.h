@@ -106,8 +106,9 @@ typedef struct svt_stats {
 typedef struct svt_plan_info {
   int num_items;                       /* attention work items of one svt_run launch */
   int splits[SVT_MAX_STREAMS];         /* KV chunks per stream (1 = no merge pass) */
-  int kv_tiles[SVT_MAX_STREAMS];       /* 128-token KV tiles per stream */
-  int64_t kv_tokens[SVT_MAX_STREAMS];  /* visible tokens per stream */
+  int kv_tiles[SVT_MAX_STREAMS];       /* KV tiles per stream (128 tokens at D = 64, 64 at
+                                          D = 128; dense-segment tiles included) */
+  int64_t kv_tokens[SVT_MAX_STREAMS];  /* visible tokens per stream (+ dense-segment rows) */
   int64_t qo_len[SVT_MAX_STREAMS];     /* query rows per stream */
 } svt_plan_info;
 
