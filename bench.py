@@ -314,7 +314,11 @@ def run_gpu(args, rank, world, local_rank):
         stream.wait_event(copied[i % 2])
         stream.wait_event(drained[i % 2])
         buf = stage[i % 2]
-        step(t0 + i, lambda b, t: buf[b], outs=outs[i % 2])
+        if args.e2e_path == "graph":   # one svt_frame_step call, replayed as a CUDA graph
+            cache.frame_step([buf[b][1] for b in range(L)], [buf[b][2] for b in range(L)],
+                             [buf[b][0] for b in range(L)], outs[i % 2], use_graph=True)
+        else:
+            step(t0 + i, lambda b, t: buf[b], outs=outs[i % 2])
         consumed[i % 2].record(stream)
         computed[i % 2].record(stream)
         enqueue_copy_out(i)
@@ -635,6 +639,9 @@ def main():
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", default="svt", choices=["svt", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--e2e-path", default="graph", choices=["graph", "calls"],
+                    help="end-to-end leg: svt_frame_step with CUDA-graph replay, or the separate "
+                         "calls of the device-resident leg")
     ap.add_argument("--workload", default=WORKLOAD, choices=sorted(PREFILL) + list(SECONDARY),
                     help="vitl_step (1 block, no RoPE) is the small case used for profiling; "
                          "tiny_stream, ragged4 and rollback10k print their own metric")
@@ -727,9 +734,12 @@ def main():
         "cpu_baseline": cpu,
         "e2e": {"value": e2e_fps, "unit": "frames/s", "h2d_bytes_per_step": r["h2d_per_step"],
                 "d2h_bytes_per_step": r["d2h_per_step"], "steps": r["e2e_steps"],
+                "path": args.e2e_path,
                 "note": f"Q/K/V of all {w.blocks} blocks copied from pinned host memory and the "
                         f"outputs of all {w.blocks} blocks copied back to pinned host memory every "
-                        "frame, on two copy streams (double-buffered by frame parity)"},
+                        "frame, on two copy streams (double-buffered by frame parity); frame step "
+                        + ("through svt_frame_step with CUDA-graph replay" if args.e2e_path == "graph"
+                           else "through the separate calls")},
         "gpu_launches": r["kernels_per_step"] * args.steps,
         "clocks": r["clocks"],
     }

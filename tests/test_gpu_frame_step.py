@@ -129,3 +129,34 @@ def test_frame_step_reports_errors_and_keeps_state():
     c.set_defer_eviction(False)
     c.frame_step([k], [v], [q], [torch.empty_like(q)])
     c.device_error()
+
+
+def test_frame_step_graph_at_full_size():
+    """The 24-block ViT-L stream with 2-D RoPE: after the steady-state
+    pre-fill, frame steps through svt_frame_step with graph replay give
+    outputs bit-identical to the separate calls for every block."""
+    from dataclasses import replace
+    w = replace(WORKLOADS["vitl_stream24"], R=2)
+    frames = w.S + w.W + 4
+    mp = max_pages_for(w, [frames])
+    a, g = make_cache(w, mp), make_cache(w, mp)
+    banks = [FrameBank(w, b, 0, need_oracle=False) for b in range(w.blocks)]
+    for t in range(w.S + w.W):
+        for c in (a, g):
+            for b in range(w.blocks):
+                c.append_frame(b, *banks[b].device(t)[1:])
+            c.evict_frames()
+    for t in range(w.S + w.W, frames):
+        ks = [banks[b].device(t)[1] for b in range(w.blocks)]
+        vs = [banks[b].device(t)[2] for b in range(w.blocks)]
+        qs = [banks[b].device(t)[0] for b in range(w.blocks)]
+        ref = _separate(a, w, ks, vs, qs)
+        got = g.frame_step(ks, vs, qs, _out_like(w, qs), use_graph=True)
+        for b in range(w.blocks):
+            assert torch.equal(got[b], ref[b]), f"t={t} block {b}"
+        for x, y in zip(a.get_page_table(), g.get_page_table()):
+            assert np.array_equal(x, y)
+    builds, replays = g.graph_counts()
+    assert builds + replays == frames - w.S - w.W and builds <= 2
+    a.device_error()
+    g.device_error()
