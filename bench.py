@@ -55,11 +55,11 @@ SECONDARY = ("tiny_stream", "ragged4", "rollback10k")
 
 # DRAM traffic of one attention launch, from an ncu capture of the single
 # ViT-L step (one 1375-row frame over 99,792 visible keys, 5 KV splits):
-# dram__bytes_read.sum 461.1 MB + dram__bytes_write.sum 25.8 MB.  Traffic
+# dram__bytes_read.sum 454.0 MB + dram__bytes_write.sum 23.4 MB.  Traffic
 # grows with the visible keys, so the bench scales it to the mean key count of
 # its timed frames.  Set to None when the attention kernel changes until a new
 # capture is taken.
-ATTN_TRAFFIC_BYTES, ATTN_TRAFFIC_KEYS = 486.82e6, 99792
+ATTN_TRAFFIC_BYTES, ATTN_TRAFFIC_KEYS = 477.37e6, 99792
 
 
 def _peaks():
