@@ -262,7 +262,9 @@ SVT_API int svt_run_extra(svt_cache* c, int block, const void* q, const void* k_
  * k, v, q, out: HOST arrays of num_blocks DEVICE pointers.  Deferred eviction applies as set by
  * svt_set_defer_eviction.  [P1] Sec. Step-by-Step Streaming Inference; [P1] Sec. Implementation
  * Examples (the upstream captures a block's forward in a CUDA graph).
- * use_graph = 0: the kernels are launched one by one, as by the separate calls.
+ * The appends of all blocks (num_blocks <= 64) share their page ids and run as one kernel
+ * launch; the pool bytes are the same as from the separate calls.
+ * use_graph = 0: the kernels are launched one by one.
  * use_graph = 1: the step's launches are recorded and issued as one CUDA graph launch.  The
  * library keeps an executable graph per launch sequence met (up to 8): the first step with a
  * new sequence builds and instantiates it, later steps give its kernel nodes the new arguments

@@ -157,6 +157,9 @@ struct svt_cache {
   // step are recorded into `rec` instead of being issued, then handed to an
   // executable graph whose kernel nodes are given the new arguments.
   Recorder* rec = nullptr;
+  // svt_frame_step gathers the appends of all blocks here and launches them
+  // together (nullptr: each svt_append_frame launches its own kernel).
+  AppendBatch* batch = nullptr;
   struct StepGraph {
     std::vector<const void*> funcs;       // kernel of each node, in launch order
     cudaGraph_t graph = nullptr;
@@ -612,6 +615,15 @@ int svt_append_frame(svt_cache* c, int block, int stream, const void* k, const v
     for (int i = 0; i < s.cur_n_sp; ++i) ap.sp_pages[i] = s.cur_sp[i];
     ap.rope_tab = c->rope_grid ? c->d_rope_tab : nullptr;
     ap.rope_grid = c->rope_grid;
+    if (c->batch) {   // launched later, with the other blocks of this frame
+      if (block == 0) c->batch->p = ap;
+      c->batch->k[block] = ap.k;
+      c->batch->v[block] = ap.v;
+      c->batch->n_blocks = block + 1;
+      s.blocks_done = block + 1;
+      if (block == 0) debug_stats(c, stream, "append");
+      return SVT_OK;
+    }
     cudaError_t e = launch_append(ap, c->dtype, reinterpret_cast<cudaStream_t>(cs), c->rec);
     if (e != cudaSuccess) {
       if (block == 0) {  // undo the allocation so that a failed call changes nothing
@@ -1052,7 +1064,34 @@ int svt_frame_step(svt_cache* c, int stream, const void* const* k, const void* c
   Recorder rec;
   c->rec = use_graph ? &rec : nullptr;
   int r = SVT_OK;
-  for (int b = 0; b < c->L && !r; ++b) r = svt_append_frame(c, b, stream, k[b], v[b], cs);
+  // The appends of all blocks share their page ids: one launch covers them.
+  if (c->L <= kMaxBatchBlocks) {
+    AppendBatch batch{};
+    batch.block_bytes = (size_t)c->max_pages * 2 * c->page_tokens * c->H * c->D * c->elem;
+    c->batch = &batch;
+    for (int b = 0; b < c->L && !r; ++b) r = svt_append_frame(c, b, stream, k[b], v[b], cs);
+    c->batch = nullptr;
+    if (r && batch.n_blocks > 0) {   // a later block was refused: undo the frame's allocation
+      const std::string msg = g_err;
+      StreamState& st = c->st[stream];
+      st.has_prov = true;
+      svt_rollback_last_frame(c, stream);
+      st.has_prov = false;
+      g_err = msg;
+    }
+    if (!r) {
+      cudaError_t e = launch_append_batch(batch, c->dtype, s, c->rec);
+      if (e != cudaSuccess) {
+        StreamState& st = c->st[stream];
+        st.has_prov = true;
+        svt_rollback_last_frame(c, stream);
+        st.has_prov = false;
+        r = cuda_fail(e, "append kernel launch");
+      }
+    }
+  } else {
+    for (int b = 0; b < c->L && !r; ++b) r = svt_append_frame(c, b, stream, k[b], v[b], cs);
+  }
   if (!r) r = svt_evict_frames(c, stream);
   if (!r) r = svt_build_visible_page_table(c, cs);
   if (!r) {

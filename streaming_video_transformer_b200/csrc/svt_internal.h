@@ -114,6 +114,19 @@ struct AppendParams {
 };
 cudaError_t launch_append(const AppendParams& p, int dtype, cudaStream_t s, Recorder* rec);
 
+// The appends of one frame for blocks 0..n_blocks-1 in one launch: the same
+// page ids for every block (p, with the block-0 mirror update), block b's pool
+// region at p.pool_block + b * block_bytes, its rows in k[b] and v[b].
+constexpr int kMaxBatchBlocks = 64;
+struct AppendBatch {
+  AppendParams p;
+  int n_blocks;
+  size_t block_bytes;
+  const char* k[kMaxBatchBlocks];
+  const char* v[kMaxBatchBlocks];
+};
+cudaError_t launch_append_batch(const AppendBatch& b, int dtype, cudaStream_t s, Recorder* rec);
+
 // ------------------------------------------------------------- RoPE on Q
 struct RopeQParams {
   const char* q_in;          // [rows][H][D]

@@ -71,15 +71,16 @@ __device__ __forceinline__ size_t pool_offset(const AppendParams& p, int kv, int
   return ((size_t)(page * 2 + kv) * p.page_tokens + off) * row_bytes;
 }
 
+// The K (kv = 0) or V (kv = 1) rows of one frame of one block, read from
+// src, scattered into that block's pool region; grid-stride over x.
 template <typename T>
-__global__ void __launch_bounds__(256) append_kernel(AppendParams p) {
-  const int kv = blockIdx.y;
-  const char* src = kv ? p.v : p.k;
+__device__ __forceinline__ void append_rows(const AppendParams& p, int kv, const char* src,
+                                            char* pool_block, bool mirror) {
   const size_t row_bytes = (size_t)p.H * p.D * sizeof(T);
   const int vpr = (int)(row_bytes / 16);              // vectors per row
   const int rows = p.ns + p.P;
   const long total = (long)rows * vpr;
-  if (kv == 0 && blockIdx.x == 0 && threadIdx.x == 0 && p.mirror_patch) {
+  if (mirror && kv == 0 && blockIdx.x == 0 && threadIdx.x == 0 && p.mirror_patch) {
     *p.mirror_patch = p.patch_page;
     for (int i = 0; i < p.n_new_sp; ++i) p.mirror_special[i] = p.new_sp[i];
   }
@@ -93,7 +94,7 @@ __global__ void __launch_bounds__(256) append_kernel(AppendParams p) {
     const int vi = (int)(i % vpr);
     const size_t dst_row = pool_offset(p, kv, row, row_bytes);
     const uint4* s = reinterpret_cast<const uint4*>(src + (size_t)row * row_bytes) + vi;
-    uint4* d = reinterpret_cast<uint4*>(p.pool_block + dst_row) + vi;
+    uint4* d = reinterpret_cast<uint4*>(pool_block + dst_row) + vi;
     if (!rope || row < p.ns) {
       *d = __ldg(s);
       continue;
@@ -111,6 +112,20 @@ __global__ void __launch_bounds__(256) append_kernel(AppendParams p) {
     d[0] = lo;
     d[half_v] = hi;
   }
+}
+
+template <typename T>
+__global__ void __launch_bounds__(256) append_kernel(AppendParams p) {
+  const int kv = blockIdx.y;
+  append_rows<T>(p, kv, kv ? p.v : p.k, p.pool_block, true);
+}
+
+// Every block's append of one frame in one launch: blockIdx.z is the block.
+template <typename T>
+__global__ void __launch_bounds__(256) append_batch_kernel(AppendBatch b) {
+  const int kv = blockIdx.y, blk = blockIdx.z;
+  append_rows<T>(b.p, kv, kv ? b.v[blk] : b.k[blk], b.p.pool_block + (size_t)blk * b.block_bytes,
+                 blk == 0);
 }
 
 template <typename T>
@@ -372,6 +387,17 @@ cudaError_t launch_append(const AppendParams& p, int dtype, cudaStream_t s, Reco
     case SVT_BF16: return dispatch(rec, append_kernel<__nv_bfloat16>, grid, 256, 0, s, p);
     case SVT_FP16: return dispatch(rec, append_kernel<__half>, grid, 256, 0, s, p);
     default: return dispatch(rec, append_kernel<float>, grid, 256, 0, s, p);
+  }
+}
+
+cudaError_t launch_append_batch(const AppendBatch& b, int dtype, cudaStream_t s, Recorder* rec) {
+  const AppendParams& p = b.p;
+  const long vecs = (long)(p.ns + p.P) * p.H * p.D * p.elem / 16;
+  dim3 grid(std::max(1, grid_for(vecs, 256) / std::max(1, b.n_blocks / 4)), 2, b.n_blocks);
+  switch (dtype) {
+    case SVT_BF16: return dispatch(rec, append_batch_kernel<__nv_bfloat16>, grid, 256, 0, s, b);
+    case SVT_FP16: return dispatch(rec, append_batch_kernel<__half>, grid, 256, 0, s, b);
+    default: return dispatch(rec, append_batch_kernel<float>, grid, 256, 0, s, b);
   }
 }
 

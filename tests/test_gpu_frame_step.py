@@ -156,6 +156,8 @@ def test_frame_step_graph_at_full_size():
             assert torch.equal(got[b], ref[b]), f"t={t} block {b}"
         for x, y in zip(a.get_page_table(), g.get_page_table()):
             assert np.array_equal(x, y)
+    # the one-launch append of all 24 blocks wrote the same pool bytes
+    assert torch.equal(a.pool, g.pool)
     builds, replays = g.graph_counts()
     assert builds + replays == frames - w.S - w.W and builds <= 2
     a.device_error()
