@@ -23,10 +23,12 @@
  *    of one cache must be issued on one CUDA stream (or ordered by the caller):
  *    kernels read the device page table written by earlier launches.  Host-side
  *    bookkeeping takes effect at call time; nothing here synchronises with the
- *    device except svt_device_error and svt_read_device_page_table.
+ *    device except svt_device_error, svt_noalloc_device_error,
+ *    svt_read_device_page_table and svt_selftest_wait_limit.
  *  - The library allocates its own device memory (page-table mirror, visible
- *    table, split-KV workspace, RoPE tables) once in svt_create_cache and frees
- *    it in svt_destroy_cache.  It never frees caller memory.
+ *    table, split-KV workspace, RoPE tables and scratch) once in
+ *    svt_create_cache and frees it in svt_destroy_cache; svt_frame_step keeps
+ *    its CUDA graphs until svt_destroy_cache.  It never frees caller memory.
  */
 #ifndef SVT_H
 #define SVT_H
