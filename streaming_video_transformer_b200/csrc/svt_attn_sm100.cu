@@ -545,12 +545,18 @@ cudaError_t launch_t(const AttnParams& p, const void* tq, const void* tkv, const
                      const void* tve, cudaStream_t s, Recorder* rec) {
   using C = Cfg<D>;
   auto kern = attn_sm100_kernel<D, BF16>;
-  static bool configured = false;
-  if (!configured) {
-    cudaError_t e =
-        cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
+  // The shared-memory opt-in is a per-device function attribute: set it once
+  // on every device the kernel is launched on.
+  constexpr int kMaxDev = 64;
+  static bool configured[kMaxDev] = {};
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= kMaxDev) return cudaErrorInvalidDevice;
+  if (!configured[dev]) {
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
     if (e != cudaSuccess) return e;
-    configured = true;
+    configured[dev] = true;
   }
   CUtensorMap mq, mkv, mke, mve;
   memcpy(&mq, tq, sizeof(mq));
