@@ -161,3 +161,27 @@ def test_noalloc_rejects_oversized_split_request():
                           num_splits=64)
     assert e.value.code == _lib.SVT_EINVAL
     assert "scratch" in str(e.value)
+
+
+def test_noalloc_on_a_pool_without_cross_frame_special():
+    """A pool whose pages hold a frame's patches followed by its specials
+    (page_size + num_special tokens per page): the allocation-free call,
+    given that page size, matches svt_run, twice in a row."""
+    w = small_workload(H=2, D=64, P=100, ns=6, S=1, W=3, dtype="bf16", R=8)
+    c = make_cache(w, w.S + w.W + 1, cross_frame_special=False)
+    bank = FrameBank(w, 0, 0, need_oracle=False)
+    for t in range(7):
+        c.append_frame(0, *bank.device(t)[1:])
+        c.evict_frames()
+    c.build_visible_page_table()
+    c.plan([w.Nq])
+    q = bank.device(6)[0]
+    ref = c.run(0, q)
+    ip, ix, lp = c.get_page_table()
+    assert list(lp) == [w.P + w.ns]
+    for call in range(2):
+        out = torch.full_like(q, float("nan"))
+        attention_noalloc(q, out, c.pool[0], torch.from_numpy(ix).to("cuda"), ip, lp, [w.Nq],
+                          c.max_pages, c.page_tokens)
+        _close(out, ref)
+    noalloc_device_error()
