@@ -50,3 +50,21 @@ def test_single_rank_passthrough():
     import bench
     assert bench.max_over_ranks([3.0, 4.0], 1, "cpu") == [3.0, 4.0]
     assert bench.whole_job_rate(1, 925, 20000.0) == pytest.approx(46.25)
+
+
+def test_timed_window_is_centred_in_the_stream():
+    """The timed frames of the 24-block stream sit in the middle of its 1000
+    frames (after the 72-frame steady-state pre-fill and the warm-up); the
+    defaults time frames 75..999; other workloads keep their pre-fill."""
+    sys.path.insert(0, ROOT)
+    import bench
+    for warmup, steps in ((3, 925), (5, 20), (3, 2), (3, 200), (5, 1000)):
+        p = bench.prefill_frames("vitl_stream24", warmup, steps)
+        first, last = p + warmup, p + warmup + steps - 1
+        assert p >= bench.PREFILL["vitl_stream24"]
+        if steps <= 925:
+            assert last <= 999
+            before = first - (bench.PREFILL["vitl_stream24"] + warmup)
+            assert abs(before - (999 - last)) <= 1
+    assert bench.prefill_frames("vitl_stream24", 3, 925) == 72
+    assert bench.prefill_frames("vitl_step", 5, 20) == bench.PREFILL["vitl_step"]
