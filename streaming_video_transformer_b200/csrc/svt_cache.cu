@@ -856,23 +856,40 @@ int svt_plan_extra(svt_cache* c, const int32_t* qo_len, const int32_t* extra_len
   // costs steers the choice), shared by the CTAs resident on one SM.
   const double tile_us = 4.0 * kTileM * TN * c->D / 6.6e6 * attn_ctas_per_sm(c->D);
   const double item_us = 2.0;
+  const int slots = c->num_sms * attn_ctas_per_sm(c->D);
+  // The KV tiles' work does not depend on the split: every chunk set covers
+  // each stream's tiles once per head and query tile.
+  double tile_work = 0;
+  for (int i = 0; i < c->n_streams; ++i)
+    if (qo_len[i]) tile_work += (double)c->H * qt[i] * tiles[i] * tile_us;
   std::vector<int> best(c->n_streams, 1);
   double best_t = 1e300;
   std::vector<double> cost;
   for (int k = 1; k <= c->max_splits; ++k) {
     std::vector<int> ch(c->n_streams, 1);
     bool split = false;
-    cost.clear();
-    double merge_bytes = 0;
+    double merge_bytes = 0, n_items = 0;
     for (int i = 0; i < c->n_streams; ++i) {
       if (!qo_len[i]) continue;
       int cc = (int)std::ceil((double)k * tiles[i] / std::max(1, max_tiles));
       cc = std::max(1, std::min({cc, c->max_splits, tiles[i]}));
       ch[i] = cc;
+      n_items += (double)c->H * cc * qt[i];
       if (cc > 1) {
         split = true;
         merge_bytes += (double)qo_len[i] * c->H * (c->D + 1) * 4.0 * (cc + 1);
       }
+    }
+    const double merge_us = split ? 4.0 + merge_bytes / 5.0e6 : 0.0;
+    // No schedule finishes before its work spread evenly over the CTA slots,
+    // and that bound never falls as k grows (more items, more merge traffic):
+    // once it reaches what the best split so far would have to beat, no
+    // larger k can be chosen.
+    if (((tile_work + n_items * item_us) / slots + merge_us) * (1.0 - 1e-9) >= best_t * 0.98) break;
+    cost.clear();
+    for (int i = 0; i < c->n_streams; ++i) {
+      if (!qo_len[i]) continue;
+      const int cc = ch[i];
       const int per_item = 1;   // one 128-row query tile per work item
       const int groups = (qt[i] + per_item - 1) / per_item;
       for (int h = 0; h < c->H; ++h)
@@ -883,8 +900,7 @@ int svt_plan_extra(svt_cache* c, const int32_t* qo_len, const int32_t* extra_len
             cost.push_back(item_us + (t1 - t0) * tile_us * q_in_item);
           }
     }
-    double t = simulate(cost, c->num_sms * attn_ctas_per_sm(c->D)) +
-               (split ? 4.0 + merge_bytes / 5.0e6 : 0.0);
+    const double t = simulate(cost, slots) + merge_us;
     if (t < best_t * 0.98) {
       best_t = t;
       best = ch;
