@@ -49,8 +49,11 @@ def prefill_frames(workload, warmup, steps):
         return base
     room = STREAM_FRAMES - base - warmup
     return base + max(0, (room - steps) // 2)
-# further workloads measured by run_secondary (one JSON line each)
-SECONDARY = ("tiny_stream", "ragged4", "rollback10k")
+# further workloads measured by run_secondary (one JSON line each), with the
+# workload whose shapes they use
+SECONDARY = {"tiny_stream": "tiny_stream", "ragged4": "ragged4", "rollback10k": "rollback10k",
+             "first_pass8": "vitl_stream24", "skip_append": "vitl_step",
+             "nocross_step": "vitl_step"}
 
 
 # DRAM traffic of one attention launch, from an ncu capture of the single
@@ -351,7 +354,15 @@ def run_secondary(args):
                    per frame), repeated; ragged4 -- one batched run over four
                    streams aged 10/70/300/2000 (fp16, D=128); rollback10k --
                    10,000 offered frames, every 3rd deferred and rejected with
-                   p=0.3, in bf16, and a sample of late frames with an fp32 pool."""
+                   p=0.3, in bf16, and a sample of late frames with an fp32 pool;
+    first_pass8 -- the first pass over the 8 scale frames of the RoPE stream
+                   (one block): all 8 x 1375 queries attend over all 8
+                   frames at once, no mask among them;
+    skip_append -- a non-keyframe of the single ViT-L step attending to the
+                   cache plus its own K/V: as a dense segment (nothing
+                   stored), and through defer, append, attend and roll back;
+    nocross_step -- the single ViT-L step on a pool without cross-frame
+                   special retention (a frame's specials leave with it)."""
     import torch
     from dataclasses import replace
 
@@ -360,7 +371,9 @@ def run_secondary(args):
 
     dev = torch.device("cuda", 0)
     torch.cuda.set_device(dev)
-    w = WORKLOADS[args.workload]
+    w = WORKLOADS[SECONDARY[args.workload]]
+    if args.workload == "first_pass8":
+        w = replace(w, blocks=1)
     ev = lambda: torch.cuda.Event(enable_timing=True)
     line = {"impl": "svt", "workload": args.workload, "n_gpus": 1, "data": "synthetic",
             "dtype": w.dtype, "config": _config(w)}
@@ -445,6 +458,120 @@ def run_secondary(args):
         line.update(metric="batched run over 4 ragged streams", value=flops / (ms / 1e3) / 1e12,
                     unit="TFLOP/s", ms_per_run=ms, kv_tokens=info["kv_tokens"],
                     splits=info["splits"], steps=args.steps)
+    elif args.workload == "first_pass8":
+        F = w.S
+        c = PagedKVCache(F + w.W + 4, w.P, w.H, w.D, w.W, w.S, num_special=w.ns, dtype=w.dtype,
+                         max_qo_len=F * w.Nq, rope_grid=w.rope_grid, rope_theta=w.rope_theta,
+                         device=dev)
+        fr = [[x.to(dev) for x in frame_qkv(w, 0, 0, t)] for t in range(F)]
+        q = torch.cat([fr[t][0] for t in range(F)])
+        out = torch.empty_like(q)
+        # the 8 frames' K/V (90 MB) fit in L2: flush it before every timed pass
+        flush = torch.empty(2 * L2_BYTES, dtype=torch.uint8, device=dev)
+
+        def first_pass():
+            c.reset()
+            for t in range(F):
+                c.append_frame(0, fr[t][1], fr[t][2])
+                c.evict_frames()
+            c.build_visible_page_table()
+            c.plan([F * w.Nq])
+            c.run(0, q, out=out)
+
+        for _ in range(args.warmup):
+            first_pass()
+        torch.cuda.synchronize()
+        whole, runs = [], []
+        for _ in range(args.steps):
+            flush.zero_()
+            a, b = ev(), ev()
+            a.record()
+            first_pass()
+            b.record()
+            flush.zero_()
+            x, y = ev(), ev()
+            x.record()
+            c.run(0, q, out=out)
+            y.record()
+            whole.append((a, b))
+            runs.append((x, y))
+        torch.cuda.synchronize()
+        nk = c.plan_info()["kv_tokens"][0]
+        flops = flops_of(F * w.Nq, nk, w.H, w.D)
+        ms_whole = statistics.median(x.elapsed_time(y) for x, y in whole)
+        ms_run = statistics.median(x.elapsed_time(y) for x, y in runs)
+        line["config"]["l2"] = "8 frames' K/V (90 MB) fit in L2; L2 flushed before each timed pass"
+        line.update(metric="attention TFLOP/s of the multi-frame first pass (8 scale frames)",
+                    value=flops / (ms_run / 1e3) / 1e12, unit="TFLOP/s", ms_run=ms_run,
+                    ms_first_pass=ms_whole, query_rows=F * w.Nq, kv_tokens=nk,
+                    splits=c.plan_info()["splits"], steps=args.steps,
+                    note="value: svt_run over all 8 frames' queries; ms_first_pass adds the 8 "
+                         "appends (with the K rotation), the table build and the plan")
+    elif args.workload in ("skip_append", "nocross_step"):
+        cross = args.workload == "skip_append"
+        pre = PREFILL["vitl_step"]
+        c = PagedKVCache(w.S + w.W + 2 + math.ceil(pre * w.ns / w.P) + 2, w.P, w.H, w.D, w.W, w.S,
+                         num_special=w.ns, dtype=w.dtype, max_qo_len=w.Nq,
+                         cross_frame_special=cross, device=dev)
+        fr = [[x.to(dev) for x in frame_qkv(w, 0, 0, i)] for i in range(w.R)]
+        for t in range(pre):
+            c.append_frame(0, fr[t % w.R][1], fr[t % w.R][2])
+            c.evict_frames()
+        c.build_visible_page_table()
+        q, k, v = fr[pre % w.R]
+        out = torch.empty_like(q)
+
+        def timed(fn):
+            for _ in range(args.warmup):
+                fn()
+            torch.cuda.synchronize()
+            marks = []
+            for _ in range(args.steps):
+                a, b = ev(), ev()
+                a.record()
+                fn()
+                b.record()
+                marks.append((a, b))
+            torch.cuda.synchronize()
+            return statistics.median(x.elapsed_time(y) for x, y in marks)
+
+        if cross:
+            def segment():
+                c.plan([w.Nq], extra_len=[w.Nq])
+                c.run(0, q, out=out, k_extra=k, v_extra=v)
+
+            def via_pool():
+                c.set_defer_eviction(True)
+                c.append_frame(0, k, v)
+                c.evict_frames()
+                c.build_visible_page_table()
+                c.plan([w.Nq])
+                c.run(0, q, out=out)
+                c.rollback_last_frame()
+                c.set_defer_eviction(False)
+                c.build_visible_page_table()
+
+            ms_seg = timed(segment)
+            c.plan([w.Nq], extra_len=[w.Nq])
+            nk = c.plan_info()["kv_tokens"][0]
+            ms_pool = timed(via_pool)
+            line.update(metric="non-keyframe step: attention over the cache plus its own K/V",
+                        value=flops_of(w.Nq, nk, w.H, w.D) / (ms_seg / 1e3) / 1e12,
+                        unit="TFLOP/s", ms_dense_segment=ms_seg, ms_defer_append_rollback=ms_pool,
+                        kv_tokens=nk, steps=args.steps,
+                        note="value: svt_plan_extra + svt_run_extra with the frame's K/V as a "
+                             "dense segment (nothing written to the pool); "
+                             "ms_defer_append_rollback: the frame appended, attended and rolled "
+                             "back (the table rebuilt afterwards)")
+        else:
+            c.plan([w.Nq])
+            nk = c.plan_info()["kv_tokens"][0]
+            ms = timed(lambda: c.run(0, q, out=out))
+            line.update(metric="single ViT-L step without cross-frame special retention",
+                        value=flops_of(w.Nq, nk, w.H, w.D) / (ms / 1e3) / 1e12, unit="TFLOP/s",
+                        ms_run=ms, kv_tokens=nk, splits=c.plan_info()["splits"],
+                        steps=args.steps)
+        line["config"]["cross_frame_special"] = cross
     else:   # rollback10k
         dec = keyframe_decisions(w, w.frames)
         n_acc = sum(1 for d, r in dec if not r)
@@ -644,7 +771,8 @@ def main():
                          "calls of the device-resident leg")
     ap.add_argument("--workload", default=WORKLOAD, choices=sorted(PREFILL) + list(SECONDARY),
                     help="vitl_step (1 block, no RoPE) is the small case used for profiling; "
-                         "tiny_stream, ragged4 and rollback10k print their own metric")
+                         "tiny_stream, ragged4, rollback10k, first_pass8, skip_append and "
+                         "nocross_step print their own metric")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
