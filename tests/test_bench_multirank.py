@@ -68,3 +68,14 @@ def test_timed_window_is_centred_in_the_stream():
             assert abs(before - (999 - last)) <= 1
     assert bench.prefill_frames("vitl_stream24", 3, 925) == 72
     assert bench.prefill_frames("vitl_step", 5, 20) == bench.PREFILL["vitl_step"]
+
+
+def test_secondary_workloads_use_defined_shapes():
+    sys.path.insert(0, ROOT)
+    import bench
+    from streaming_video_transformer_b200.inputs import WORKLOADS
+    assert set(bench.PREFILL) <= set(WORKLOADS)
+    for name, base in bench.SECONDARY.items():
+        assert base in WORKLOADS, name
+    # the rows of the scope table each have a measurement line
+    assert {"first_pass8", "skip_append", "nocross_step", "tiny_stream"} <= set(bench.SECONDARY)
