@@ -31,8 +31,10 @@
 //               has completed (which also leaves O quiescent for a rescale),
 //               and recomputes the tile against its exact maximum only when
 //               the row sum of P_j exceeds 2^8 (always on the first tile).
-// The exponential unit is the bound at D = 64 (one exp per 256 MMA flops);
-// the two CTAs on an SM keep it busy between each other's phases.
+// At D = 64 a tile needs twice as many exponential-unit cycles as tensor
+// cycles (one exp per 256 MMA flops), but the measured limit is the latency of
+// each CTA's S -> softmax -> P -> P.V chain; the two CTAs on an SM overlap
+// their chains.
 // Split-KV chunks write fp32 partials and LSE; a merge kernel combines them.
 
 #include <cuda.h>
