@@ -123,18 +123,58 @@ def _visible(t, w):
 
 
 class ClockSampler:
-    """nvidia-smi clocks / throttle reasons sampled during the timed region."""
+    """SM clock, power and clock-event (throttle) reasons sampled during the
+    timed region: read through NVML every 20 ms on the device the run uses
+    (found by its UUID), else with nvidia-smi every 200 ms.  Read-only: no
+    setting of the GPU is touched."""
 
     FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    # NVML clock-event reason bits
+    REASON_BITS = {"sw_power_cap": 0x4, "hw_slowdown": 0x8, "sw_thermal_slowdown": 0x20,
+                   "hw_thermal_slowdown": 0x40}
+    INTERVAL_S = 0.02
 
     def __init__(self, device_index):
         self.idx = device_index
         self.proc = None
         self.path = None
+        self.thread = None
+        self.rows = []
+        self.max_mhz = None
+
+    def _nvml_handle(self):
+        import pynvml
+        import torch
+        pynvml.nvmlInit()
+        uuid = str(torch.cuda.get_device_properties(self.idx).uuid)
+        if not uuid.startswith("GPU-"):
+            uuid = "GPU-" + uuid
+        return pynvml, pynvml.nvmlDeviceGetHandleByUUID(uuid.encode())
+
+    def _poll(self, nv, h):
+        get_reasons = getattr(nv, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
+            nv.nvmlDeviceGetCurrentClocksThrottleReasons
+        while not self.stop.is_set():
+            try:
+                self.rows.append((nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM),
+                                  nv.nvmlDeviceGetPowerUsage(h) / 1000.0, int(get_reasons(h))))
+            except Exception:
+                pass
+            self.stop.wait(self.INTERVAL_S)
 
     def __enter__(self):
+        try:
+            import threading
+            nv, h = self._nvml_handle()
+            self.max_mhz = nv.nvmlDeviceGetMaxClockInfo(h, nv.NVML_CLOCK_SM)
+            self.stop = threading.Event()
+            self.thread = threading.Thread(target=self._poll, args=(nv, h), daemon=True)
+            self.thread.start()
+            return self
+        except Exception:
+            self.thread = None
         try:
             fd, self.path = tempfile.mkstemp(suffix=".csv")
             os.close(fd)
@@ -147,6 +187,9 @@ class ClockSampler:
         return self
 
     def __exit__(self, *exc):
+        if self.thread is not None:
+            self.stop.set()
+            self.thread.join(timeout=5)
         if self.proc is not None:
             self.proc.terminate()
             try:
@@ -156,6 +199,16 @@ class ClockSampler:
             self.out.close()
 
     def summary(self):
+        if self.thread is not None:
+            if not self.rows:
+                return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": ["no samples"],
+                        "source": "nvml"}
+            reasons = sorted({n for _, _, bits in self.rows
+                              for n, b in self.REASON_BITS.items() if bits & b})
+            return {"sm_mhz": statistics.median(r[0] for r in self.rows),
+                    "sm_max_mhz": self.max_mhz, "reasons": reasons, "samples": len(self.rows),
+                    "power_w_max": max(r[1] for r in self.rows),
+                    "source": f"nvml every {int(self.INTERVAL_S * 1000)} ms"}
         if self.proc is None or not self.path:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unavailable"]}
         rows = []
@@ -175,7 +228,8 @@ class ClockSampler:
                 "sm_max_mhz": max(mx) if mx else None, "reasons": reasons,
                 "samples": len(rows),
                 "power_w_max": max((float(r[3]) for r in rows
-                                    if r[3].replace(".", "").isdigit()), default=None)}
+                                    if r[3].replace(".", "").isdigit()), default=None),
+                "source": "nvidia-smi every 200 ms"}
 
 
 # ------------------------------------------------------------------ GPU arm
