@@ -143,6 +143,7 @@ class ClockSampler:
         self.thread = None
         self.rows = []
         self.max_mhz = None
+        self.limit_w = None
 
     def _nvml_handle(self):
         import pynvml
@@ -169,6 +170,10 @@ class ClockSampler:
             import threading
             nv, h = self._nvml_handle()
             self.max_mhz = nv.nvmlDeviceGetMaxClockInfo(h, nv.NVML_CLOCK_SM)
+            try:
+                self.limit_w = nv.nvmlDeviceGetEnforcedPowerLimit(h) / 1000.0
+            except Exception:
+                self.limit_w = None
             self.stop = threading.Event()
             self.thread = threading.Thread(target=self._poll, args=(nv, h), daemon=True)
             self.thread.start()
@@ -208,6 +213,7 @@ class ClockSampler:
             return {"sm_mhz": statistics.median(r[0] for r in self.rows),
                     "sm_max_mhz": self.max_mhz, "reasons": reasons, "samples": len(self.rows),
                     "power_w_max": max(r[1] for r in self.rows),
+                    "power_limit_w": self.limit_w,
                     "source": f"nvml every {int(self.INTERVAL_S * 1000)} ms"}
         if self.proc is None or not self.path:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unavailable"]}
