@@ -252,7 +252,10 @@ def run_gpu(args, rank, world, local_rank):
     w = replace(WORKLOADS[args.workload], R=4)
     L = w.blocks
     prefill = prefill_frames(args.workload, args.warmup, args.steps)
-    e2e_steps = min(args.steps, max(8, args.steps // 4))
+    # The end-to-end leg's first copy in and last copy out cannot overlap
+    # compute; as many frames as the device-resident leg (8 to 64) keep
+    # that fill and drain from dominating a short run.
+    e2e_steps = min(max(args.steps, 8), 64)
     total_frames = prefill + args.warmup + args.steps + e2e_steps
     max_pages = (w.S + w.W + 1) + math.ceil(total_frames * w.ns / w.P) + 2
     cache = PagedKVCache(max_pages, w.P, w.H, w.D, w.W, w.S, num_blocks=L, num_special=w.ns,
