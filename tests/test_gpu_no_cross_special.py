@@ -11,6 +11,7 @@ import golden_io
 from alloc_model import AllocModel
 from gpu_util import (FrameBank, assert_close, gather_visible, make_cache, oracle_out,
                       oracle_stream_for)
+from oracle import attend_lse
 from streaming_video_transformer_b200.inputs import WORKLOADS, small_workload
 
 pytestmark = pytest.mark.gpu
@@ -164,4 +165,39 @@ def test_vitl_step_full_size_without_retention():
     gk, gv = gather_visible(c, 0, 0)
     ok, ov = st.visible_kv()
     assert np.array_equal(gk, ok) and np.array_equal(gv, ov)
+    c.device_error()
+
+
+@pytest.mark.parametrize("cfg", [
+    dict(P=122, ns=6, S=1, W=3, H=2, D=64, frames=7),                       # 128-token pages
+    dict(P=100, ns=6, S=1, W=2, H=2, D=128, frames=5, rope_grid=10),        # D = 128, RoPE
+])
+def test_dense_segment_without_retention(cfg):
+    """A non-keyframe attends through a dense K/V segment on a pool whose
+    pages hold a frame's patches and specials: the segment's tiles follow
+    the pages' (page_size + num_special)-token tiles; nothing is stored."""
+    w = small_workload(**cfg, R=cfg["frames"] + 1)
+    c = make_cache(w, _pages(w), cross_frame_special=False)
+    bank = FrameBank(w, 0, 0)
+    st = oracle_stream_for(c, w)
+    for t in range(w.frames):
+        _frame(c, w, bank, t)
+        st.append_frame(*bank.oracle(t)[1:])
+    c.build_visible_page_table()
+    table, stats = c.get_page_table(), c.get_cache_stats()
+    pool0 = c.pool.clone()
+    q, k, v = bank.device(w.frames)
+    c.plan([w.Nq], extra_len=[w.Nq])
+    assert c.plan_info()["kv_tokens"][0] == st.num_visible_tokens() + w.Nq
+    out = c.run(0, q, k_extra=k, v_extra=v)
+    out32 = c.run(0, q, k_extra=k, v_extra=v, force_fp32=True)
+    q64, k64, v64 = bank.oracle(w.frames)
+    kc, vc = st.visible_kv()
+    ref, _ = attend_lse(q64, np.concatenate([kc, k64]), np.concatenate([vc, v64]))
+    assert_close(out, ref, what="segment")
+    assert_close(out32, ref, fp32=True, what="segment fp32")
+    assert torch.equal(c.pool, pool0)
+    for a, b in zip(table, c.get_page_table()):
+        assert np.array_equal(a, b)
+    assert c.get_cache_stats() == stats
     c.device_error()
