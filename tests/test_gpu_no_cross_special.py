@@ -201,3 +201,59 @@ def test_dense_segment_without_retention(cfg):
         assert np.array_equal(a, b)
     assert c.get_cache_stats() == stats
     c.device_error()
+
+
+def test_frame_step_graph_without_retention():
+    """svt_frame_step with graph replay on a pool without retention (two
+    blocks, the batched append writing each frame's specials after its
+    patches): outputs, tables and pool bytes equal the separate calls'."""
+    w = small_workload(P=40, ns=6, S=2, W=3, H=2, D=64, frames=10, R=10, blocks=2)
+    a = make_cache(w, _pages(w), cross_frame_special=False)
+    g = make_cache(w, _pages(w), cross_frame_special=False)
+    banks = [FrameBank(w, b, 0, need_oracle=(b == 0)) for b in range(w.blocks)]
+    st = oracle_stream_for(a, w)
+    for t in range(w.frames):
+        ks = [banks[b].device(t)[1] for b in range(w.blocks)]
+        vs = [banks[b].device(t)[2] for b in range(w.blocks)]
+        qs = [banks[b].device(t)[0] for b in range(w.blocks)]
+        for b in range(w.blocks):
+            a.append_frame(b, ks[b], vs[b])
+        a.evict_frames()
+        a.build_visible_page_table()
+        a.plan([w.Nq])
+        ref = [a.run(b, qs[b]) for b in range(w.blocks)]
+        got = g.frame_step(ks, vs, qs, [torch.empty_like(q) for q in qs], use_graph=True)
+        for b in range(w.blocks):
+            assert torch.equal(got[b], ref[b]), f"t={t} block {b}"
+        for x, y in zip(a.get_page_table(), g.get_page_table()):
+            assert np.array_equal(x, y)
+        st.append_frame(*banks[0].oracle(t)[1:])
+        o, _ = oracle_out(st, banks[0].oracle(t)[0])
+        assert_close(got[0], o, what=f"t={t + 1}")
+    assert torch.equal(a.pool, g.pool)
+    builds, replays = g.graph_counts()
+    assert builds + replays == w.frames and replays >= w.frames - 3
+    a.device_error()
+    g.device_error()
+
+
+def test_multi_frame_first_pass_without_retention():
+    """Three frames appended, then all of their queries attend at once over
+    the frames' patches and specials (no mask among them), with RoPE."""
+    w = small_workload(P=36, ns=6, S=4, W=4, H=2, D=64, R=8, rope_grid=6)
+    F = 3
+    c = make_cache(w, _pages(w), cross_frame_special=False, max_qo_len=F * w.Nq)
+    bank = FrameBank(w, 0, 0)
+    st = oracle_stream_for(c, w)
+    for t in range(F):
+        _frame(c, w, bank, t)
+        st.append_frame(*bank.oracle(t)[1:])
+    c.build_visible_page_table()
+    c.plan([F * w.Nq])
+    assert c.plan_info()["kv_tokens"][0] == st.num_visible_tokens() == F * w.Nq
+    q = torch.cat([bank.device(t)[0] for t in range(F)])
+    q64 = np.concatenate([bank.oracle(t)[0] for t in range(F)])
+    ref, _ = oracle_out(st, q64)
+    assert_close(c.run(0, q), ref, what="first pass")
+    assert_close(c.run(0, q, force_fp32=True), ref, fp32=True, what="first pass fp32")
+    c.device_error()
