@@ -162,3 +162,41 @@ def test_frame_step_graph_at_full_size():
     assert builds + replays == frames - w.S - w.W and builds <= 2
     a.device_error()
     g.device_error()
+
+
+def test_frame_step_on_the_second_stream_of_a_shared_pool():
+    """Two streams in one pool: stream 0 holds history, frame steps (graph
+    replay) run on stream 1; outputs and tables equal the separate calls',
+    and stream 0's part of the table is untouched."""
+    w = small_workload(P=16, ns=6, S=2, W=3, H=2, D=64, frames=9, R=9, blocks=2)
+    mp = max_pages_for(w, [w.frames, w.frames], num_streams=2)
+    a, g = make_cache(w, mp, num_streams=2), make_cache(w, mp, num_streams=2)
+    b0 = [FrameBank(w, b, 0, need_oracle=False) for b in range(w.blocks)]
+    b1 = [FrameBank(w, b, 1, need_oracle=(b == 0)) for b in range(w.blocks)]
+    for c in (a, g):
+        for t in range(5):
+            for b in range(w.blocks):
+                c.append_frame(b, *b0[b].device(t)[1:], stream=0)
+            c.evict_frames(0)
+    st = oracle_stream(w)
+    for t in range(w.frames):
+        ks = [b1[b].device(t)[1] for b in range(w.blocks)]
+        vs = [b1[b].device(t)[2] for b in range(w.blocks)]
+        qs = [b1[b].device(t)[0] for b in range(w.blocks)]
+        for b in range(w.blocks):
+            a.append_frame(b, ks[b], vs[b], stream=1)
+        a.evict_frames(1)
+        a.build_visible_page_table()
+        a.plan([0, w.Nq])
+        ref = [a.run(b, qs[b]) for b in range(w.blocks)]
+        got = g.frame_step(ks, vs, qs, _out_like(w, qs), stream=1, use_graph=True)
+        for b in range(w.blocks):
+            assert torch.equal(got[b], ref[b]), f"t={t} block {b}"
+        for x, y in zip(a.get_page_table(), g.get_page_table()):
+            assert np.array_equal(x, y)
+        st.append_frame(*b1[0].oracle(t)[1:])
+        o, _ = oracle_out(st, b1[0].oracle(t)[0])
+        assert_close(got[0], o, what=f"stream 1 t={t + 1}")
+    assert torch.equal(a.pool, g.pool)
+    a.device_error()
+    g.device_error()

@@ -257,3 +257,27 @@ def test_multi_frame_first_pass_without_retention():
     assert_close(c.run(0, q), ref, what="first pass")
     assert_close(c.run(0, q, force_fp32=True), ref, fp32=True, what="first pass fp32")
     c.device_error()
+
+
+def test_two_streams_batched_without_retention():
+    """Two streams of different ages in one pool without retention, one
+    batched run: each stream's rows against its own oracle stream."""
+    w = small_workload(P=60, ns=6, S=2, W=3, H=2, D=64, R=12)
+    ages = [4, 11]
+    c = make_cache(w, 2 * _pages(w), num_streams=2, cross_frame_special=False)
+    banks = [FrameBank(w, 0, s) for s in range(2)]
+    sts = [oracle_stream_for(c, w) for _ in range(2)]
+    for s, age in enumerate(ages):
+        for t in range(age):
+            _frame(c, w, banks[s], t, stream=s)
+            sts[s].append_frame(*banks[s].oracle(t)[1:])
+    c.build_visible_page_table()
+    c.plan([w.Nq, w.Nq])
+    q = torch.cat([banks[s].device(ages[s] - 1)[0] for s in range(2)])
+    out = c.run(0, q)
+    out32 = c.run(0, q, force_fp32=True)
+    for s in range(2):
+        ref, _ = oracle_out(sts[s], banks[s].oracle(ages[s] - 1)[0])
+        assert_close(out[s * w.Nq:(s + 1) * w.Nq], ref, what=f"stream {s}")
+        assert_close(out32[s * w.Nq:(s + 1) * w.Nq], ref, fp32=True, what=f"fp32 stream {s}")
+    c.device_error()
