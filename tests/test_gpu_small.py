@@ -9,6 +9,7 @@ from alloc_model import AllocModel
 from gpu_util import (FrameBank, assert_close, gather_visible, make_cache, max_pages_for,
                       oracle_out, oracle_stream)
 from oracle import attend_lse
+from streaming_video_transformer_b200 import _lib
 from streaming_video_transformer_b200.inputs import WORKLOADS, frame_qkv, small_workload
 
 pytestmark = pytest.mark.gpu
@@ -397,4 +398,51 @@ def test_skip_append_with_dense_segment(cfg):
     c.plan([w.Nq, 0])
     ref, _ = oracle_out(sts[0], banks[0].oracle(8)[0])
     assert_close(c.run(0, banks[0].device(8)[0]), ref, what="frame after the segment step")
+    c.device_error()
+
+
+def test_dense_segment_on_a_stream_with_no_stored_frames():
+    """The first frame of a stream attended as a non-keyframe: no pages are
+    visible and every KV tile comes from the dense segment (bf16 and fp32
+    paths, D = 64 and D = 128); the table stays empty."""
+    for D, P in ((64, 200), (128, 100)):
+        w = small_workload(P=P, ns=6, S=2, W=3, H=2, D=D, R=2)
+        c = make_cache(w, max_pages_for(w, [2]))
+        c.build_visible_page_table()
+        q, k, v = FrameBank(w, 0, 0).device(0)
+        q64, k64, v64 = FrameBank(w, 0, 0).oracle(0)
+        c.plan([w.Nq], extra_len=[w.Nq])
+        info = c.plan_info()
+        assert info["kv_tokens"][0] == w.Nq
+        ref, _ = attend_lse(q64, k64, v64)
+        assert_close(c.run(0, q, k_extra=k, v_extra=v), ref, what=f"D={D}")
+        assert_close(c.run(0, q, k_extra=k, v_extra=v, force_fp32=True), ref, fp32=True,
+                     what=f"fp32 D={D}")
+        ip, ix, lp = c.get_page_table()
+        assert list(ip) == [0, 0] and len(ix) == 0
+        c.device_error()
+
+
+def test_batch_of_the_maximum_number_of_streams():
+    """SVT_MAX_STREAMS (32) streams of different ages in one pool and one
+    batched run; sampled streams against the oracle."""
+    w = small_workload(P=16, ns=6, S=1, W=2, H=2, D=64, R=6)
+    n = _lib.MAX_STREAMS
+    ages = [1 + (s % 6) for s in range(n)]
+    c = make_cache(w, max_pages_for(w, ages, num_streams=n), num_streams=n)
+    banks = [FrameBank(w, 0, s, need_oracle=(s % 7 == 0)) for s in range(n)]
+    sts = {s: oracle_stream(w) for s in range(0, n, 7)}
+    for s, age in enumerate(ages):
+        for t in range(age):
+            c.append_frame(0, *banks[s].device(t)[1:], stream=s)
+            c.evict_frames(s)
+            if s in sts:
+                sts[s].append_frame(*banks[s].oracle(t)[1:])
+    c.build_visible_page_table()
+    c.plan([w.Nq] * n)
+    q = torch.cat([banks[s].device(ages[s] - 1)[0] for s in range(n)])
+    out = c.run(0, q)
+    for s, st in sts.items():
+        ref, _ = oracle_out(st, banks[s].oracle(ages[s] - 1)[0])
+        assert_close(out[s * w.Nq:(s + 1) * w.Nq], ref, what=f"stream {s}")
     c.device_error()

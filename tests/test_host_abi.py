@@ -301,3 +301,17 @@ def test_plan_tiles_items_and_split_bounds(D, tile):
         assert 1 <= info["splits"][s] <= min(8, tiles)
         items += H * -(-qo[s] // 128) * info["splits"][s]
     assert info["num_items"] == items
+
+
+def test_binding_constants_match_the_header():
+    """The binding's copies of the header's constants (status codes, dtypes,
+    the stream limit that sizes svt_plan_info's arrays)."""
+    import re
+    hdr = open(os.path.join(ROOT, "include", "svt.h")).read()
+    m = re.search(r"#define SVT_MAX_STREAMS (\d+)", hdr)
+    assert m and int(m.group(1)) == _lib.MAX_STREAMS
+    for name in ("SVT_OK", "SVT_EINVAL", "SVT_ENOPAGES", "SVT_ESTATE", "SVT_ECUDA", "SVT_EDEVICE",
+                 "SVT_BF16", "SVT_FP16", "SVT_FP32"):
+        m = re.search(name + r"\s*=\s*(-?\d+)", hdr)
+        assert m, name
+        assert int(m.group(1)) == getattr(_lib, name), name
